@@ -1,0 +1,358 @@
+/*
+ * CPU oracle for the NVFP4 block-scaled GEMM -- plain, slow, obviously
+ * correct.  TEST INFRASTRUCTURE ONLY (see nvfp4_oracle.h): the CUDA library
+ * never includes or links this file, and this file includes nothing of it.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * (no FMA contraction and IEEE float semantics are part of the quantizer's
+ * definition, since its integer codes are compared bit for bit).
+ *
+ * Sources (the three pages):
+ *   [P1] "The SM120 FP4 Kernel Disaster", section "Input Knowledge Required",
+ *        item 3: FP4 packs two 4-bit values per byte, with per-block scales.
+ *   [P3] "Peeling the Kernel Onion", section "The Benchmark Design": FP8 scale
+ *        factors one per 16 elements, BF16 output, bytes
+ *        M*K/2 + K*N/2 + M*K/16 + K*N/16 + 2*M*N.
+ *   [P3c] "Peeling the Kernel Onion", section "The Chain of Reasoning": the
+ *        FP4 GEMM takes a global alpha and writes an out tensor.
+ * The element format (E2M1: 1 sign, 2 exponent, 1 mantissa bit, values
+ * {0,0.5,1,1.5,2,3,4,6}) and the scale format (E4M3: bias 7, no infinities,
+ * NaN at S.1111.111) are the standard NVFP4 definitions these pages use.
+ */
+#include "nvfp4_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef __int128 i128;
+typedef unsigned __int128 u128;
+
+/* ------------------------------------------------------------------------ */
+/* Format tables                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* E2M1 magnitudes, code bits 2..0 (exponent bits 2..1, mantissa bit 0). */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_value(int code) {
+    code &= 0xF;
+    double m = E2M1_MAG[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* E4M3 (bias 7): exponent field e = bits 6..3, mantissa m = bits 2..0.
+ * e == 0: subnormal m * 2^-9;  otherwise (1 + m/8) * 2^(e-7);
+ * e == 15 && m == 7: NaN.  No infinities. */
+double oracle_e4m3_value(int byte) {
+    byte &= 0xFF;
+    int s = byte >> 7, e = (byte >> 3) & 0xF, m = byte & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else        v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Integer forms used by the exact accumulation.
+ * e2m1 magnitude in units of 1/2; e4m3 magnitude in units of 2^-9. */
+static int e2m1_half_units(int code) { return (int)(E2M1_MAG[code & 7] * 2.0); }
+static int e4m3_units(int byte) { return (int)ldexp(fabs(oracle_e4m3_value(byte)), 9); }
+
+/* Round-to-nearest, ties to the even code, over a monotone table of
+ * non-negative values val[0..n-1]; values at or above val[n-1] saturate to
+ * code n-1 (the "satfinite" behaviour). */
+static int round_nearest_even(double v, const double* val, int n) {
+    if (v >= val[n - 1]) return n - 1;
+    int c = 0;
+    while (c + 1 < n && val[c + 1] <= v) c++;      /* val[c] <= v < val[c+1] */
+    double mid = (val[c] + val[c + 1]) * 0.5;       /* exact: few significant bits */
+    if (v < mid) return c;
+    if (v > mid) return c + 1;
+    return (c & 1) ? c + 1 : c;                     /* tie: even code */
+}
+
+static double E4M3_POS[127];   /* codes 0x00..0x7E */
+static int e4m3_pos_ready = 0;
+static void init_e4m3_pos(void) {
+    if (e4m3_pos_ready) return;
+    for (int c = 0; c < 127; c++) E4M3_POS[c] = oracle_e4m3_value(c);
+    e4m3_pos_ready = 1;
+}
+
+int oracle_e4m3_rne_satfinite(float v) {
+    init_e4m3_pos();
+    if (isnan(v)) return 0x7F;
+    int sign = signbit(v) ? 0x80 : 0;
+    return sign | round_nearest_even(fabs((double)v), E4M3_POS, 127);
+}
+
+int oracle_e2m1_rne_satfinite(float v) {
+    if (isnan(v)) return -1;
+    int sign = signbit(v) ? 8 : 0;
+    return sign | round_nearest_even(fabs((double)v), E2M1_MAG, 8);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantize-and-pack                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Per tensor: g = amax / (6 * 448).  Per 16-element K block:
+ * s = E4M3_rne_satfinite(amax_blk / (6 * g)); each element
+ * q = E2M1_rne_satfinite(x / (g * decode(s))), packed two per byte with the
+ * even-k element in the low nibble.  All arithmetic in IEEE fp32. */
+int oracle_quantize(const float* X, int rows, int K,
+                    uint8_t* codes, uint8_t* scales, float* g_out) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
+    float amax = 0.0f;
+    for (long i = 0; i < (long)rows * K; i++) {
+        if (!isfinite(X[i])) return -1;
+        float a = fabsf(X[i]);
+        if (a > amax) amax = a;
+    }
+    /* An all-zero tensor has no scale to recover; g = 1 keeps every step finite. */
+    volatile float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    volatile float six_g = 6.0f * g;
+    for (int r = 0; r < rows; r++) {
+        const float* x = X + (long)r * K;
+        uint8_t* crow = codes + (long)r * (K / 2);
+        uint8_t* srow = scales + (long)r * (K / 16);
+        memset(crow, 0, (size_t)(K / 2));
+        for (int b = 0; b < K / 16; b++) {
+            float amax_blk = 0.0f;
+            for (int i = 0; i < 16; i++) {
+                float a = fabsf(x[b * 16 + i]);
+                if (a > amax_blk) amax_blk = a;
+            }
+            volatile float t = amax_blk / six_g;
+            int s = oracle_e4m3_rne_satfinite(t);
+            srow[b] = (uint8_t)s;
+            volatile float denom = g * (float)oracle_e4m3_value(s);
+            for (int i = 0; i < 16; i++) {
+                int k = b * 16 + i;
+                int q;
+                if (denom == 0.0f) {
+                    q = signbit(x[k]) ? 8 : 0;   /* a zero scale carries zero codes */
+                } else {
+                    volatile float v = x[k] / denom;
+                    q = oracle_e2m1_rne_satfinite(v);
+                }
+                crow[k / 2] |= (uint8_t)((k & 1) ? (q << 4) : q);
+            }
+        }
+    }
+    *g_out = g;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Exact rounding of alpha * S * 2^-20 to BF16                              */
+/* ------------------------------------------------------------------------ */
+
+static int bitlen_u128(u128 x) {
+    int n = 0;
+    while (x) { n++; x >>= 1; }
+    return n;
+}
+
+/* BF16: 8 significant bits, exponent bias 127, subnormals in steps of 2^-133. */
+static uint16_t bf16_rne_of(i128 S, float alpha) {
+    uint32_t ab;
+    memcpy(&ab, &alpha, 4);
+    int sign_a = (int)(ab >> 31), ea = (int)((ab >> 23) & 0xFF);
+    uint32_t fa = ab & 0x7FFFFF;
+    if (ea == 0xFF) {                       /* alpha is inf or NaN */
+        if (fa || S == 0) return 0x7FC0;
+        return (uint16_t)((((S < 0) ^ sign_a) << 15) | 0x7F80);
+    }
+    uint32_t ma = ea ? (fa | 0x800000u) : fa;
+    int E = (ea ? ea - 150 : -149) - 20;    /* value = |S| * ma * 2^E */
+    if (S == 0 || ma == 0) return 0x0000;   /* an exact zero is reported as +0 */
+    int sign = (S < 0) ^ sign_a;
+    u128 P = (u128)(S < 0 ? -S : S) * (u128)ma;
+    int nb = bitlen_u128(P);
+    int ev = nb - 1 + E;                    /* 2^ev <= value < 2^(ev+1) */
+    int shift = (ev >= -126) ? nb - 8 : (-133 - E);
+    u128 q;
+    if (shift > 0) {
+        q = P >> shift;
+        u128 rem = P - (q << shift), half = (u128)1 << (shift - 1);
+        if (rem > half || (rem == half && (q & 1))) q++;
+    } else {
+        q = P << (-shift);
+    }
+    int eq = E + shift;                     /* value ~= q * 2^eq */
+    if (q == 256) { q = 128; eq += 1; }
+    uint16_t bits;
+    if (q >= 128) {
+        int biased = eq + 7 + 127;
+        if (biased >= 255) bits = 0x7F80;   /* overflow rounds to infinity */
+        else bits = (uint16_t)((biased << 7) | (int)(q - 128));
+    } else {
+        bits = (uint16_t)q;                 /* subnormal (eq == -133) or zero */
+    }
+    return (uint16_t)((sign << 15) | bits);
+}
+
+uint16_t oracle_bf16_of_scaled(int64_t s_hi, uint64_t s_lo, float alpha) {
+    i128 S = (i128)(((u128)(uint64_t)s_hi << 64) | (u128)s_lo);
+    return bf16_rne_of(S, alpha);
+}
+
+/* ------------------------------------------------------------------------ */
+/* The GEMM                                                                 */
+/* ------------------------------------------------------------------------ */
+
+static int scales_valid(const uint8_t* s, long n) {
+    for (long i = 0; i < n; i++)
+        if ((s[i] & 0x80) || s[i] == 0x7F) return 0;   /* unsigned, non-NaN */
+    return 1;
+}
+
+/* Decode one packed row into signed integers a_k in units of 2^-10:
+ * a_k = e2m1(code_k) * e4m3(scale_{k/16}); code_k is the low nibble of
+ * byte k/2 for even k and the high nibble for odd k. */
+static void decode_row(const uint8_t* codes, const uint8_t* scales, int K, int32_t* out) {
+    for (int k = 0; k < K; k++) {
+        int c = (k & 1) ? (codes[k / 2] >> 4) : (codes[k / 2] & 0xF);
+        int v = e2m1_half_units(c) * e4m3_units(scales[k / 16]);
+        out[k] = (c & 8) ? -v : v;
+    }
+}
+
+/* Sum_k a_k b_k exactly (units 2^-20), with the fp64 sum in the same order as
+ * a cross-check; returns the BF16 of alpha * sum and the fp64 views. */
+static uint16_t dot_decoded(const int32_t* a, const int32_t* b, int K, float alpha,
+                            double* exact, double* absdot) {
+    i128 S = 0, A = 0;
+    double Sd = 0.0;
+    for (int k = 0; k < K; k++) {
+        int64_t t = (int64_t)a[k] * (int64_t)b[k];
+        S += t;
+        A += (t < 0 ? -t : t);
+        Sd += (double)t;
+    }
+    /* fp64 is exact while every partial sum stays below 2^53 units. */
+    if (A < ((i128)1 << 53) && (i128)Sd != S) abort();
+    if (exact) *exact = ldexp((double)S, -20) * (double)alpha;
+    if (absdot) *absdot = ldexp((double)A, -20) * fabs((double)alpha);
+    return bf16_rne_of(S, alpha);
+}
+
+uint16_t oracle_dot(const uint8_t* a_row, const uint8_t* sa_row,
+                    const uint8_t* b_row, const uint8_t* sb_row,
+                    int K, float alpha, double* exact, double* absdot) {
+    int32_t* a = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+    int32_t* b = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+    decode_row(a_row, sa_row, K, a);
+    decode_row(b_row, sb_row, K, b);
+    uint16_t r = dot_decoded(a, b, K, alpha, exact, absdot);
+    free(a);
+    free(b);
+    return r;
+}
+
+static int gemm_args_ok(int M, int N, int K) {
+    return M >= 0 && N >= 0 && K > 0 && K % 16 == 0 && K <= (1 << 20);
+}
+
+int oracle_gemm(const uint8_t* A, const uint8_t* sA,
+                const uint8_t* B, const uint8_t* sB,
+                float alpha, int M, int N, int K,
+                uint16_t* D_bf16, double* ref, double* absdot) {
+    if (!gemm_args_ok(M, N, K)) return -1;
+    if (!scales_valid(sA, (long)M * (K / 16)) || !scales_valid(sB, (long)N * (K / 16))) return -1;
+    int32_t* a = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+    int32_t* bdec = (int32_t*)malloc(sizeof(int32_t) * (size_t)K * (size_t)(N > 0 ? N : 1));
+    for (int n = 0; n < N; n++)
+        decode_row(B + (long)n * (K / 2), sB + (long)n * (K / 16), K, bdec + (long)n * K);
+    for (int m = 0; m < M; m++) {
+        decode_row(A + (long)m * (K / 2), sA + (long)m * (K / 16), K, a);
+        for (int n = 0; n < N; n++) {
+            double e, ad;
+            uint16_t d = dot_decoded(a, bdec + (long)n * K, K, alpha, &e, &ad);
+            long o = (long)m * N + n;
+            if (D_bf16) D_bf16[o] = d;
+            if (ref) ref[o] = e;
+            if (absdot) absdot[o] = ad;
+        }
+    }
+    free(a);
+    free(bdec);
+    return 0;
+}
+
+int oracle_gemm_sampled(const uint8_t* A, const uint8_t* sA,
+                        const uint8_t* B, const uint8_t* sB,
+                        float alpha, int M, int N, int K,
+                        const int32_t* rows, const int32_t* cols, int count,
+                        uint16_t* D_bf16, double* ref, double* absdot) {
+    if (!gemm_args_ok(M, N, K) || count < 0) return -1;
+    for (int i = 0; i < count; i++) {
+        int m = rows[i], n = cols[i];
+        if (m < 0 || m >= M || n < 0 || n >= N) return -1;
+        if (!scales_valid(sA + (long)m * (K / 16), K / 16) ||
+            !scales_valid(sB + (long)n * (K / 16), K / 16)) return -1;
+        double e, ad;
+        uint16_t d = oracle_dot(A + (long)m * (K / 2), sA + (long)m * (K / 16),
+                                B + (long)n * (K / 2), sB + (long)n * (K / 16),
+                                K, alpha, &e, &ad);
+        if (D_bf16) D_bf16[i] = d;
+        if (ref) ref[i] = e;
+        if (absdot) absdot[i] = ad;
+    }
+    return 0;
+}
+
+int oracle_grouped_gemm(const uint8_t* A, const uint8_t* sA,
+                        const uint8_t* B, const uint8_t* sB,
+                        const float* alpha, const int32_t* row_offsets, int G,
+                        int M_total, int N, int K,
+                        uint16_t* D_bf16, double* ref, double* absdot) {
+    if (!gemm_args_ok(M_total, N, K) || G < 0) return -1;
+    if (row_offsets[0] != 0 || row_offsets[G] != M_total) return -1;
+    for (int g = 0; g < G; g++)
+        if (row_offsets[g + 1] < row_offsets[g]) return -1;
+    for (int g = 0; g < G; g++) {
+        int r0 = row_offsets[g], rows = row_offsets[g + 1] - r0;
+        if (rows == 0) continue;
+        long o = (long)r0 * N;
+        int rc = oracle_gemm(A + (long)r0 * (K / 2), sA + (long)r0 * (K / 16),
+                             B + (long)g * N * (K / 2), sB + (long)g * N * (K / 16),
+                             alpha[g], rows, N, K,
+                             D_bf16 ? D_bf16 + o : NULL, ref ? ref + o : NULL,
+                             absdot ? absdot + o : NULL);
+        if (rc) return rc;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scale-factor layout for the tensor cores                                 */
+/* ------------------------------------------------------------------------ */
+
+/* One 512-byte atom holds 128 rows x 4 consecutive scale blocks (one MMA K
+ * step of 64 elements): row r, block j of the atom sits at byte
+ * 16*(r%32) + 4*(r/32) + j.  Atoms follow each other along K, then along
+ * 128-row blocks. */
+long oracle_swizzled_bytes(int rows, int K) {
+    if (rows < 0 || K <= 0 || K % 64 != 0) return -1;
+    long row_blocks = (rows + 127) / 128;
+    return row_blocks * (K / 64) * 512L;
+}
+
+int oracle_swizzle_scales(const uint8_t* s, int rows, int K, uint8_t* out) {
+    long bytes = oracle_swizzled_bytes(rows, K);
+    if (bytes < 0) return -1;
+    int kb_per_row = K / 16, steps = K / 64;
+    long row_blocks = (rows + 127) / 128;
+    for (long r = 0; r < row_blocks * 128; r++) {
+        for (int kb = 0; kb < kb_per_row; kb++) {
+            uint8_t v = (r < rows) ? s[r * kb_per_row + kb] : 0;
+            long rb = r / 128, rr = r % 128, step = kb / 4, j = kb % 4;
+            long off = (rb * steps + step) * 512 + 16 * (rr % 32) + 4 * (rr / 32) + j;
+            out[off] = v;
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,91 @@
+/*
+ * CPU oracle for the NVFP4 block-scaled GEMM.  TEST INFRASTRUCTURE ONLY:
+ * only the tests, the smoke check and the benchmark's CPU-baseline leg may
+ * call it.  The product path never includes, links or executes anything in
+ * this directory, and this directory shares no code with the CUDA library.
+ *
+ * What it computes (all citations are to the three source pages):
+ *   - NVFP4 data: 4-bit E2M1 values packed two per byte, with a scale factor
+ *     per block of values ("The SM120 FP4 Kernel Disaster", section "Input
+ *     Knowledge Required", item 3).
+ *   - One FP8 (E4M3) block scale per 16 elements along K, BF16 output; the
+ *     byte model M*K/2 + K*N/2 + M*K/16 + K*N/16 + 2*M*N ("Peeling the Kernel
+ *     Onion", section "The Benchmark Design").
+ *   - A global fp32 scale alpha applied to the output ("Peeling the Kernel
+ *     Onion", section "The Chain of Reasoning": the kernel needs alpha).
+ *
+ *   D[m][n] = bf16_rne( alpha * sum_k e2m1(A[m,k]) * e4m3(sA[m,k/16])
+ *                                  * e2m1(B[n,k]) * e4m3(sB[n,k/16]) )
+ *
+ * The sum is formed exactly (128-bit integer fixed point in units of 2^-20,
+ * cross-checked against fp64), alpha is applied exactly, and the result is
+ * rounded once to BF16 with round-to-nearest-even.
+ *
+ * Parity status of every function is stated beside it; all are pinned by the
+ * not-gpu tests (format tables, closed forms, brute force, invariants).
+ */
+#ifndef NVFP4_ORACLE_H
+#define NVFP4_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Format tables. */
+double oracle_e2m1_value(int code);          /* code 0..15, bit 3 = sign            */
+double oracle_e4m3_value(int byte);          /* 0..255; NaN for 0x7F and 0xFF       */
+int    oracle_e4m3_rne_satfinite(float v);   /* nearest E4M3, ties to even, |v|>448 -> 448 */
+int    oracle_e2m1_rne_satfinite(float v);   /* nearest E2M1, ties to even, |v|>6 -> 6     */
+
+/* Quantize fp32 X[rows][K] to packed codes [rows][K/2], scales [rows][K/16]
+ * and one global scale g for the whole tensor.  Returns 0 on success, -1 on a
+ * bad argument (K not a multiple of 16, NaN/Inf input). */
+int oracle_quantize(const float* X, int rows, int K,
+                    uint8_t* codes, uint8_t* scales, float* g_out);
+
+/* Exact value of one output: sets *exact (double rounding of the exact
+ * value), *absdot = |alpha| * sum_k |a_k b_k| (fp64) and returns the BF16 bits
+ * of the single RNE rounding of the exact value. */
+uint16_t oracle_dot(const uint8_t* a_row, const uint8_t* sa_row,
+                    const uint8_t* b_row, const uint8_t* sb_row,
+                    int K, float alpha, double* exact, double* absdot);
+
+/* Full GEMM.  A [M][K/2], sA [M][K/16], B [N][K/2], sB [N][K/16], all
+ * row-major bytes.  D_bf16 [M][N] (may be NULL), ref [M][N] and absdot [M][N]
+ * (either may be NULL).  Returns 0, or -1 on bad arguments. */
+int oracle_gemm(const uint8_t* A, const uint8_t* sA,
+                const uint8_t* B, const uint8_t* sB,
+                float alpha, int M, int N, int K,
+                uint16_t* D_bf16, double* ref, double* absdot);
+
+/* Only the listed outputs (rows[i], cols[i]), i < count. */
+int oracle_gemm_sampled(const uint8_t* A, const uint8_t* sA,
+                        const uint8_t* B, const uint8_t* sB,
+                        float alpha, int M, int N, int K,
+                        const int32_t* rows, const int32_t* cols, int count,
+                        uint16_t* D_bf16, double* ref, double* absdot);
+
+/* Grouped GEMM: rows [off[g], off[g+1]) of A use B[g], sB[g] and alpha[g].
+ * B [G][N][K/2], sB [G][N][K/16]. */
+int oracle_grouped_gemm(const uint8_t* A, const uint8_t* sA,
+                        const uint8_t* B, const uint8_t* sB,
+                        const float* alpha, const int32_t* row_offsets, int G,
+                        int M_total, int N, int K,
+                        uint16_t* D_bf16, double* ref, double* absdot);
+
+/* BF16 RNE of the exact value alpha * S * 2^-20 (S a signed 128-bit integer
+ * given as hi:lo words).  Exposed for the rounding pins. */
+uint16_t oracle_bf16_of_scaled(int64_t s_hi, uint64_t s_lo, float alpha);
+
+/* Tensor-core scale-factor layout: row-major [rows][K/16] -> 512-byte atoms
+ * of 128 rows x 4 scale blocks, atoms ordered K-fastest within each 128-row
+ * block; padding rows are zero.  Writes oracle_swizzled_bytes() bytes. */
+long oracle_swizzled_bytes(int rows, int K);
+int  oracle_swizzle_scales(const uint8_t* s_rowmajor, int rows, int K, uint8_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
