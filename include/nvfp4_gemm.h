@@ -1,0 +1,170 @@
+/*
+ * nvfp4_gemm.h -- C ABI of the B200 (sm_100a) NVFP4 block-scaled GEMM library
+ * (libnvfp4gemm.so).
+ *
+ * The operation (one GEMM):
+ *
+ *   D[m][n] = bf16_rne( alpha * sum_k  e2m1(A[m,k]) * e4m3(sA[m, k/16])
+ *                                     * e2m1(B[n,k]) * e4m3(sB[n, k/16]) )
+ *
+ * Sources: NVFP4 packs two 4-bit values per byte with per-block scale factors
+ * ("The SM120 FP4 Kernel Disaster", section "Input Knowledge Required",
+ * item 3); one FP8 scale per 16 elements and a BF16 output, with the byte
+ * model M*K/2 + K*N/2 + M*K/16 + K*N/16 + 2*M*N ("Peeling the Kernel Onion",
+ * section "The Benchmark Design"); the call takes a global alpha and an
+ * output tensor ("Peeling the Kernel Onion", section "The Chain of
+ * Reasoning"); packed-K shapes must agree between operands ("The SM120 FP4
+ * Kernel Disaster", section "The Bash Command").
+ *
+ * Data layout at the ABI (all row-major, K the contiguous dimension):
+ *   A   uint8 [M][K/2]   E2M1 codes, element k of a row in byte k/2, the even
+ *                        k in the low nibble (bits 3..0), bit 3 of a code is
+ *                        its sign.
+ *   sA  uint8 [M][K/16]  E4M3 block scales (bias 7), one per 16 elements of a
+ *                        row.  Must be non-negative and not NaN (0x7F); this
+ *                        is not checked.
+ *   B   uint8 [N][K/2],  sB uint8 [N][K/16]   the same for the N operand ("TN").
+ *   D   bf16  [M][N].
+ * Any re-layout of the scales for the tensor cores happens on the device
+ * inside these calls.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers (cudaMalloc'd or equivalent) on the current
+ *     device unless a parameter says otherwise; the caller owns them and they
+ *     must stay valid until the work on `stream` has finished.  The library
+ *     never frees caller memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous: they enqueue work and return without
+ *     synchronising, except nvfp4_get_device_error.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns a status and launches nothing.  No exception or
+ *     abort crosses this boundary.
+ *   - The library owns per-device, per-stream scratch (re-laid-out scales,
+ *     split-K partial sums) which it allocates on first need and grows; the
+ *     first call of a new, larger shape on a stream may therefore call
+ *     cudaMalloc, so make it before capturing that stream into a CUDA graph.
+ *     Calls on different streams use different scratch and may overlap.
+ *   - Device-side waits are bounded; a wait that runs out records
+ *     NVFP4_ERR_TIMEOUT in a device error word read by nvfp4_get_device_error.
+ *   - Requires an sm_100 device (B200/GB200); others get
+ *     NVFP4_ERR_UNSUPPORTED_DEVICE.  There is no fallback path.
+ */
+#ifndef NVFP4_GEMM_H
+#define NVFP4_GEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, misaligned pointer */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 64 != 0, N % 8 != 0, size limits */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 3, /* not compute capability 10.0 */
+    NVFP4_ERR_CUDA = 4,               /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_TIMEOUT = 5,            /* a bounded device-side wait ran out */
+    NVFP4_ERR_NO_MEMORY = 6           /* scratch allocation failed */
+} nvfp4_status;
+
+/*
+ * nvfp4_gemm -- single NVFP4 GEMM, D = alpha * A * B^T (see the top of this
+ * file for the formula and layouts).
+ *   A [M][K/2], sA [M][K/16], B [N][K/2], sB [N][K/16]: device, read only.
+ *   alpha: fp32 global scale (for quantised inputs, gA * gB).
+ *   D [M][N] bf16: device, written.
+ *   Requirements: M >= 0, N >= 0, K > 0; K % 64 == 0; N % 8 == 0; A, B, D
+ *   16-byte aligned; sA, sB 4-byte aligned.  M == 0 or N == 0 is a no-op.
+ * Small M uses the weight-streaming kernel (B rows on the tensor cores' M
+ * side, split-K over the SMs); large M uses 128 x N-tile output tiles.
+ */
+nvfp4_status nvfp4_gemm(const void* A, const void* sA,
+                        const void* B, const void* sB,
+                        float alpha, void* D,
+                        int M, int N, int K, void* stream);
+
+/*
+ * nvfp4_grouped_gemm -- MoE-style grouped GEMM: G independent problems that
+ * share N and K.  Rows [row_offsets[g], row_offsets[g+1]) of A are multiplied
+ * by B[g] and scaled by alpha[g]:
+ *   D[m][n] = bf16_rne(alpha[g] * sum_k A[m,k] sA[m,k/16] B[g][n,k] sB[g][n,k/16]).
+ *   A [M_total][K/2], sA [M_total][K/16]  rows grouped by g (device).
+ *   B [G][N][K/2],    sB [G][N][K/16]     one weight matrix per group (device).
+ *   alpha [G] fp32 (device), row_offsets [G+1] int32 (device): row_offsets[0]
+ *   must be 0, row_offsets[G] must be M_total and the sequence non-decreasing
+ *   (this is not checked on the device; violating it is undefined).
+ *   D [M_total][N] bf16 (device).
+ *   Groups with no rows cost nothing and their B is never read.
+ *   Same requirements as nvfp4_gemm, and G >= 1.
+ * Sources: MoE routing gives each expert about 16 rows ("Peeling the Kernel
+ * Onion", section "The Critical Connection to Real Inference"); persistent
+ * grouped GEMM kernels amortise small per-expert problems (same page, section
+ * "Knowledge Created and Its Impact").
+ */
+nvfp4_status nvfp4_grouped_gemm(const void* A, const void* sA,
+                                const void* B, const void* sB,
+                                const float* alpha, const int32_t* row_offsets,
+                                int G, void* D,
+                                int M_total, int N, int K, void* stream);
+
+/*
+ * nvfp4_quantize -- fp32 X [rows][K] (device) to NVFP4:
+ *   g = amax(|X|) / (6 * 448)  (one global scale for the whole tensor; 1.0 if
+ *   X is all zero), per 16-element block s = E4M3_rne_satfinite(amax_blk /
+ *   (6 g)), per element q = E2M1_rne_satfinite(x / (g * s)); a zero scale
+ *   gives zero codes.  All steps IEEE fp32 with round-to-nearest-even, so the
+ *   output is bit-reproducible.  The sign of x is kept in the code, also when
+ *   it rounds to zero.
+ *   codes [rows][K/2] uint8, scales [rows][K/16] uint8, g_out [1] fp32: device,
+ *   written.  X must be finite (not checked).  K % 16 == 0, X 16-byte aligned.
+ */
+nvfp4_status nvfp4_quantize(const float* X, int rows, int K,
+                            void* codes, void* scales, float* g_out, void* stream);
+
+/*
+ * nvfp4_swizzle_scales -- re-lay row-major E4M3 scales [rows][K/16] into the
+ * tensor-core scale-factor layout the GEMM kernels feed to tcgen05.cp:
+ * 512-byte atoms of 128 rows x 4 scale blocks (one 64-element MMA K step),
+ * row r, block j of an atom at byte 16*(r%32) + 4*(r/32) + j, atoms ordered
+ * along K within each 128-row block, padding rows zero.
+ *   s_rowmajor (device, read), s_swizzled (device, nvfp4_swizzled_scale_bytes
+ *   bytes, written).  K % 64 == 0; both pointers 4-byte aligned.
+ */
+nvfp4_status nvfp4_swizzle_scales(const void* s_rowmajor, int rows, int K,
+                                  void* s_swizzled, void* stream);
+
+/* Bytes nvfp4_swizzle_scales writes: ceil(rows/128) * (K/64) * 512, or 0 for
+ * invalid arguments. */
+size_t nvfp4_swizzled_scale_bytes(int rows, int K);
+
+/*
+ * nvfp4_get_device_error -- synchronise `stream`, then read and clear the
+ * current device's error word.  Returns NVFP4_ERR_TIMEOUT if a device-side
+ * wait ran out since the last call, NVFP4_ERR_CUDA if the synchronisation
+ * failed, else NVFP4_OK.
+ */
+nvfp4_status nvfp4_get_device_error(void* stream);
+
+/* Human-readable name of a status (static storage, never NULL). */
+const char* nvfp4_status_string(nvfp4_status status);
+
+/*
+ * nvfp4_debug_wait_timeout -- diagnostics for the bounded-wait machinery:
+ * launches one block whose thread waits on a shared-memory barrier that
+ * nothing ever arrives on, using the same bounded wait as the GEMM kernels
+ * with a limit of `timeout_ns` nanoseconds (1e3 .. 5e9).  The kernel then
+ * records NVFP4_ERR_TIMEOUT in the device error word and returns normally, so
+ * a following nvfp4_get_device_error reports NVFP4_ERR_TIMEOUT and the
+ * context stays usable.
+ */
+nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_GEMM_H */

@@ -1,0 +1,192 @@
+"""NVFP4 block-scaled GEMM for NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/nvfp4_gemm.h``
+(``libnvfp4gemm.so``): it checks tensor shapes and dtypes, passes raw device
+pointers and the current CUDA stream, and raises on a non-OK status.  Every
+step of the computation runs in the library's CUDA kernels; PyTorch is used
+only for device memory and streams.  There is no CPU fallback: if the library
+is missing, importing the binding's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4gemm.so")
+
+STATUS = {
+    0: "NVFP4_OK",
+    1: "NVFP4_ERR_INVALID_ARG",
+    2: "NVFP4_ERR_UNSUPPORTED_SHAPE",
+    3: "NVFP4_ERR_UNSUPPORTED_DEVICE",
+    4: "NVFP4_ERR_CUDA",
+    5: "NVFP4_ERR_TIMEOUT",
+    6: "NVFP4_ERR_NO_MEMORY",
+}
+
+# Every symbol include/nvfp4_gemm.h declares.
+EXPORTS = (
+    "nvfp4_gemm", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
+    "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
+    "nvfp4_debug_wait_timeout", "nvfp4_version",
+)
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnvfp4gemm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m nvfp4_block_scaled_gemm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.nvfp4_gemm.argtypes = [P, P, P, P, f32, P, i32, i32, i32, P]
+        L.nvfp4_grouped_gemm.argtypes = [P, P, P, P, P, P, i32, P, i32, i32, i32, P]
+        L.nvfp4_quantize.argtypes = [P, i32, i32, P, P, P, P]
+        L.nvfp4_swizzle_scales.argtypes = [P, i32, i32, P, P]
+        L.nvfp4_swizzled_scale_bytes.argtypes = [i32, i32]
+        L.nvfp4_swizzled_scale_bytes.restype = ctypes.c_size_t
+        L.nvfp4_get_device_error.argtypes = [P]
+        L.nvfp4_status_string.argtypes = [i32]
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        L.nvfp4_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
+        for name in ("nvfp4_gemm", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
+                     "nvfp4_get_device_error", "nvfp4_debug_wait_timeout"):
+            getattr(L, name).restype = i32
+        L.nvfp4_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise Nvfp4Error(status, where)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def packed_k(a: torch.Tensor) -> int:
+    """K of a packed E2M1 tensor [rows, K/2]."""
+    return a.shape[-1] * 2
+
+
+def gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, alpha: float,
+         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """D[M,N] (bf16) = alpha * (A * sA) @ (B * sB)^T.
+
+    A uint8 [M, K/2], sA uint8 [M, K/16], B uint8 [N, K/2], sB uint8 [N, K/16].
+    K is given by the packed operands: both must hold K/2 bytes per row
+    (a mismatch is reported here rather than as a kernel error).
+    """
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D packed E2M1 tensors [rows, K/2]")
+    M, N, K = A.shape[0], B.shape[0], packed_k(A)
+    if packed_k(B) != K:
+        raise ValueError(f"K mismatch: A holds K={K} (shape {tuple(A.shape)}), B holds K={packed_k(B)} "
+                         f"(shape {tuple(B.shape)}); both operands are [rows, K/2] bytes")
+    _need(A, "A", torch.uint8, (M, K // 2))
+    _need(B, "B", torch.uint8, (N, K // 2))
+    _need(sA, "sA", torch.uint8, (M, K // 16))
+    _need(sB, "sB", torch.uint8, (N, K // 16))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _need(out, "out", torch.bfloat16, (M, N))
+    _check(lib().nvfp4_gemm(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
+                            out.data_ptr(), M, N, K, _stream(stream)), "nvfp4_gemm")
+    return out
+
+
+def grouped_gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, alpha: torch.Tensor,
+                 row_offsets: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Grouped GEMM: rows [off[g], off[g+1]) of A times B[g]^T, scaled by alpha[g].
+
+    A uint8 [M_total, K/2], sA [M_total, K/16], B uint8 [G, N, K/2],
+    sB [G, N, K/16], alpha fp32 [G], row_offsets int32 [G+1] (all CUDA).
+    """
+    if A.dim() != 2 or B.dim() != 3:
+        raise ValueError("A must be [M_total, K/2] and B [G, N, K/2]")
+    Mt, (G, N, _), K = A.shape[0], B.shape, packed_k(A)
+    if B.shape[2] * 2 != K:
+        raise ValueError(f"K mismatch: A holds K={K}, B holds K={B.shape[2] * 2}")
+    _need(A, "A", torch.uint8, (Mt, K // 2))
+    _need(sA, "sA", torch.uint8, (Mt, K // 16))
+    _need(B, "B", torch.uint8, (G, N, K // 2))
+    _need(sB, "sB", torch.uint8, (G, N, K // 16))
+    _need(alpha, "alpha", torch.float32, (G,))
+    _need(row_offsets, "row_offsets", torch.int32, (G + 1,))
+    if out is None:
+        out = torch.empty((Mt, N), dtype=torch.bfloat16, device=A.device)
+    _need(out, "out", torch.bfloat16, (Mt, N))
+    _check(lib().nvfp4_grouped_gemm(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), alpha.data_ptr(),
+                                    row_offsets.data_ptr(), G, out.data_ptr(), Mt, N, K, _stream(stream)),
+           "nvfp4_grouped_gemm")
+    return out
+
+
+def quantize(X: torch.Tensor, stream=None):
+    """fp32 [rows, K] (CUDA) -> (codes uint8 [rows, K/2], scales uint8 [rows, K/16], g fp32 [1])."""
+    if X.dim() != 2:
+        raise ValueError("X must be 2-D [rows, K]")
+    rows, K = X.shape
+    _need(X, "X", torch.float32, (rows, K))
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((rows, K // 16), dtype=torch.uint8, device=X.device)
+    g = torch.empty((1,), dtype=torch.float32, device=X.device)
+    _check(lib().nvfp4_quantize(X.data_ptr(), rows, K, codes.data_ptr(), scales.data_ptr(), g.data_ptr(),
+                                _stream(stream)), "nvfp4_quantize")
+    return codes, scales, g
+
+
+def swizzled_scale_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_swizzled_scale_bytes(rows, K))
+
+
+def swizzle_scales(s: torch.Tensor, K: int, stream=None) -> torch.Tensor:
+    """Row-major E4M3 scales [rows, K/16] -> tensor-core atom layout (flat uint8)."""
+    rows = s.shape[0]
+    _need(s, "s", torch.uint8, (rows, K // 16))
+    out = torch.empty((swizzled_scale_bytes(rows, K),), dtype=torch.uint8, device=s.device)
+    _check(lib().nvfp4_swizzle_scales(s.data_ptr(), rows, K, out.data_ptr(), _stream(stream)),
+           "nvfp4_swizzle_scales")
+    return out
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(lib().nvfp4_get_device_error(_stream(stream)))
+
+
+def debug_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check(lib().nvfp4_debug_wait_timeout(int(timeout_ns), _stream(stream)), "nvfp4_debug_wait_timeout")
+
+
+def version() -> int:
+    return int(lib().nvfp4_version())

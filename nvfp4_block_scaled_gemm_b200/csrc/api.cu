@@ -1,0 +1,382 @@
+// C ABI of libnvfp4gemm.so (declared in include/nvfp4_gemm.h): host-side
+// validation, scratch management, TMA descriptor creation and dispatch to the
+// sm_100a kernels.  All arithmetic of the GEMM happens in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/nvfp4_gemm.h"
+#include "aux_kernels.cuh"
+#include "gemm_kernel.cuh"
+
+namespace {
+
+using nvfp4::GemmParams;
+using nvfp4::TileConfig;
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// ------------------------------------------------------------ device checks
+struct DeviceInfo {
+    bool checked = false;
+    bool supported = false;
+    int num_sms = 0;
+    unsigned smem_attr_set = 0;  // bit per kernel instantiation
+};
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_devices;
+
+nvfp4_status current_device(int* dev, DeviceInfo** info) {
+    if (cudaGetDevice(dev) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_devices[*dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        d.checked = true;
+        d.supported = (major == 10 && minor == 0);
+        d.num_sms = sms;
+    }
+    *info = &d;
+    return d.supported ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED_DEVICE;
+}
+
+// ------------------------------------------------------------ scratch
+// Per (device, stream) scratch.  Layout: [split-K tile counters, kCounterBytes,
+// zero between launches][everything else].
+constexpr size_t kCounterBytes = 16384;
+constexpr int kMaxCounters = (int)(kCounterBytes / sizeof(unsigned));
+
+struct Scratch {
+    uint8_t* ptr = nullptr;
+    size_t cap = 0;
+};
+std::map<std::pair<int, uintptr_t>, Scratch> g_scratch;
+
+nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    Scratch& s = g_scratch[{dev, reinterpret_cast<uintptr_t>(stream)}];
+    if (s.cap < bytes) {
+        size_t want = std::max(bytes, s.cap * 2);
+        want = (want + 0xFFFFF) & ~size_t(0xFFFFF);
+        if (s.ptr != nullptr) {
+            // Only this stream uses this buffer: once its queue drains, it is free.
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+            cudaFree(s.ptr);
+            s.ptr = nullptr;
+            s.cap = 0;
+        }
+        void* p = nullptr;
+        if (cudaMalloc(&p, want) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_NO_MEMORY;
+        }
+        if (cudaMemsetAsync(p, 0, kCounterBytes, stream) != cudaSuccess) {
+            cudaFree(p);
+            return NVFP4_ERR_CUDA;
+        }
+        s.ptr = static_cast<uint8_t*>(p);
+        s.cap = want;
+    }
+    *out = s.ptr;
+    return NVFP4_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D map over a row-major byte matrix [rows][row_bytes]; box 128 bytes x
+// box_rows, 128-byte swizzle, zero fill out of bounds.
+bool make_operand_map(CUtensorMap* map, const void* base, long long rows, long long row_bytes, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    const cuuint32_t elem_strides[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+nvfp4_status launch_swizzle(const void* s, int rows, int K, void* out, cudaStream_t stream) {
+    const int steps = K / 64;
+    const long long lines = (long long)((rows + 127) / 128) * steps * 32;
+    if (lines == 0) return NVFP4_OK;
+    const int threads = 256;
+    const long long blocks = (lines + threads - 1) / threads;
+    nvfp4::swizzle_scales_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        static_cast<const uint8_t*>(s), rows, K / 16, steps, lines, static_cast<uint8_t*>(out));
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ GEMM dispatch
+struct Plan {
+    bool swap;
+    int bq;
+    int tiles_p, tiles_q;
+    int splits, k_tiles, k_per_split;
+};
+
+Plan make_plan(int M, int N, int K, int num_sms) {
+    Plan p{};
+    p.k_tiles = (K + 255) / 256;
+    if (M <= 128) {
+        p.swap = true;
+        p.bq = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+        p.tiles_p = (N + 127) / 128;
+        p.tiles_q = 1;
+    } else {
+        p.swap = false;
+        p.bq = N >= 256 ? 256 : 128;
+        p.tiles_p = (M + 127) / 128;
+        p.tiles_q = (N + p.bq - 1) / p.bq;
+    }
+    const int tiles = p.tiles_p * p.tiles_q;
+    int splits = 1;
+    if (tiles < num_sms && tiles <= kMaxCounters) splits = std::max(1, std::min(p.k_tiles, num_sms / tiles));
+    p.k_per_split = (p.k_tiles + splits - 1) / splits;
+    p.splits = (p.k_tiles + p.k_per_split - 1) / p.k_per_split;
+    return p;
+}
+
+template <int BQ, bool SWAP, bool SPLITK>
+nvfp4_status launch_gemm_kernel(DeviceInfo* info, unsigned bit, const CUtensorMap& tmP, const CUtensorMap& tmQ,
+                                const GemmParams& prm, dim3 grid, cudaStream_t stream) {
+    using C = TileConfig<BQ>;
+    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(info->smem_attr_set & bit)) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            info->smem_attr_set |= bit;
+        }
+    }
+    kern<<<grid, nvfp4::kThreads, C::SMEM_BYTES, stream>>>(tmP, tmQ, prm);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+template <bool SWAP, bool SPLITK>
+nvfp4_status launch_by_bq(int bq, DeviceInfo* info, const CUtensorMap& tmP, const CUtensorMap& tmQ,
+                          const GemmParams& prm, dim3 grid, cudaStream_t stream) {
+    const unsigned base = (SWAP ? 1u : 0u) * 10u + (SPLITK ? 5u : 0u);
+    switch (bq) {
+        case 16: return launch_gemm_kernel<16, SWAP, SPLITK>(info, 1u << (base + 0), tmP, tmQ, prm, grid, stream);
+        case 32: return launch_gemm_kernel<32, SWAP, SPLITK>(info, 1u << (base + 1), tmP, tmQ, prm, grid, stream);
+        case 64: return launch_gemm_kernel<64, SWAP, SPLITK>(info, 1u << (base + 2), tmP, tmQ, prm, grid, stream);
+        case 128: return launch_gemm_kernel<128, SWAP, SPLITK>(info, 1u << (base + 3), tmP, tmQ, prm, grid, stream);
+        case 256: return launch_gemm_kernel<256, SWAP, SPLITK>(info, 1u << (base + 4), tmP, tmQ, prm, grid, stream);
+        default: return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    }
+}
+
+nvfp4_status check_gemm_args(const void* A, const void* sA, const void* B, const void* sB, const void* D, int M,
+                             int N, int K) {
+    if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!A || !sA || !B || !sB || !D) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) || !aligned(sB, 4))
+        return NVFP4_ERR_INVALID_ARG;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_version(void) { return kVersion; }
+
+const char* nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "NVFP4_OK";
+        case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+        case NVFP4_ERR_UNSUPPORTED_SHAPE: return "NVFP4_ERR_UNSUPPORTED_SHAPE";
+        case NVFP4_ERR_UNSUPPORTED_DEVICE: return "NVFP4_ERR_UNSUPPORTED_DEVICE";
+        case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+        case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
+        case NVFP4_ERR_NO_MEMORY: return "NVFP4_ERR_NO_MEMORY";
+    }
+    return "NVFP4_ERR_UNKNOWN";
+}
+
+size_t nvfp4_swizzled_scale_bytes(int rows, int K) {
+    if (rows < 0 || K <= 0 || K % 64 != 0) return 0;
+    return (size_t)((rows + 127) / 128) * (size_t)(K / 64) * 512u;
+}
+
+nvfp4_status nvfp4_swizzle_scales(const void* s, int rows, int K, void* out, void* stream) {
+    if (rows < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0) return NVFP4_OK;
+    if (!s || !out || !aligned(s, 4) || !aligned(out, 16)) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    return launch_swizzle(s, rows, K, out, static_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_quantize(const float* X, int rows, int K, void* codes, void* scales, float* g_out,
+                            void* stream_) {
+    if (rows < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!g_out || (rows > 0 && (!X || !codes || !scales))) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (!aligned(X, 16) || !aligned(codes, 8))) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(g_out, 4)) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (cudaMemsetAsync(g_out, 0, sizeof(float), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const long long n = (long long)rows * K;
+    if (n > 0) {
+        const long long n4 = n / 4;
+        const int threads = 256;
+        const int blocks = (int)std::min<long long>((n4 + threads - 1) / threads, (long long)info->num_sms * 8);
+        nvfp4::amax_kernel<<<std::max(blocks, 1), threads, 0, stream>>>(reinterpret_cast<const float4*>(X), n4,
+                                                                        reinterpret_cast<unsigned*>(g_out));
+        const long long nb = n / 16;
+        nvfp4::quantize_kernel<<<(unsigned)((nb + threads - 1) / threads), threads, 0, stream>>>(
+            X, nb, reinterpret_cast<const unsigned*>(g_out), static_cast<uint8_t*>(codes),
+            static_cast<uint8_t*>(scales));
+    }
+    nvfp4::finalize_global_scale_kernel<<<1, 1, 0, stream>>>(g_out);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_gemm(const void* A, const void* sA, const void* B, const void* sB, float alpha, void* D, int M,
+                        int N, int K, void* stream_) {
+    nvfp4_status st = check_gemm_args(A, sA, B, sB, D, M, N, K);
+    if (st != NVFP4_OK || M == 0 || N == 0) return st;
+    int dev;
+    DeviceInfo* info;
+    st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+    const Plan plan = make_plan(M, N, K, info->num_sms);
+    const void* P = plan.swap ? B : A;
+    const void* Q = plan.swap ? A : B;
+    const void* sP = plan.swap ? sB : sA;
+    const void* sQ = plan.swap ? sA : sB;
+    const int rows_p = plan.swap ? N : M;
+    const int rows_q = plan.swap ? M : N;
+
+    const size_t sfp_bytes = nvfp4_swizzled_scale_bytes(rows_p, K);
+    const size_t sfq_bytes = nvfp4_swizzled_scale_bytes(rows_q, K);
+    const size_t part_bytes =
+        plan.splits > 1 ? (size_t)plan.splits * plan.tiles_p * plan.tiles_q * 128 * plan.bq * sizeof(float) : 0;
+    const size_t off_sfp = kCounterBytes;
+    const size_t off_sfq = align_up(off_sfp + sfp_bytes, 256);
+    const size_t off_part = align_up(off_sfq + sfq_bytes, 256);
+    uint8_t* ws = nullptr;
+    st = get_scratch(dev, stream, off_part + part_bytes, &ws);
+    if (st != NVFP4_OK) return st;
+
+    if ((st = launch_swizzle(sP, rows_p, K, ws + off_sfp, stream)) != NVFP4_OK) return st;
+    if ((st = launch_swizzle(sQ, rows_q, K, ws + off_sfq, stream)) != NVFP4_OK) return st;
+
+    CUtensorMap tmP, tmQ;
+    if (!make_operand_map(&tmP, P, rows_p, K / 2, 128) || !make_operand_map(&tmQ, Q, rows_q, K / 2, plan.bq))
+        return NVFP4_ERR_CUDA;
+
+    GemmParams prm{};
+    prm.sfp = ws + off_sfp;
+    prm.sfq = ws + off_sfq;
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.partials = reinterpret_cast<float*>(ws + off_part);
+    prm.counters = reinterpret_cast<unsigned*>(ws);
+    prm.alpha = alpha;
+    prm.rows_p = rows_p;
+    prm.rows_q = rows_q;
+    prm.K = K;
+    prm.ldd = N;
+    prm.k_tiles = plan.k_tiles;
+    prm.k_tiles_per_split = plan.k_per_split;
+    const dim3 grid(plan.tiles_q, plan.tiles_p, plan.splits);
+    if (plan.swap) {
+        return plan.splits > 1 ? launch_by_bq<true, true>(plan.bq, info, tmP, tmQ, prm, grid, stream)
+                               : launch_by_bq<true, false>(plan.bq, info, tmP, tmQ, prm, grid, stream);
+    }
+    return plan.splits > 1 ? launch_by_bq<false, true>(plan.bq, info, tmP, tmQ, prm, grid, stream)
+                           : launch_by_bq<false, false>(plan.bq, info, tmP, tmQ, prm, grid, stream);
+}
+
+nvfp4_status nvfp4_grouped_gemm(const void* A, const void* sA, const void* B, const void* sB, const float* alpha,
+                                const int32_t* row_offsets, int G, void* D, int M_total, int N, int K,
+                                void* stream_) {
+    if (G < 1) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_gemm_args(A, sA, B, sB, D, M_total, N, K);
+    if (st != NVFP4_OK) return st;
+    if (M_total == 0 || N == 0) return NVFP4_OK;
+    if (!alpha || !row_offsets || !aligned(alpha, 4) || !aligned(row_offsets, 4)) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    (void)stream_;
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+}
+
+nvfp4_status nvfp4_get_device_error(void* stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, nvfp4::g_error_word, sizeof(v)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(nvfp4::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    return (v & nvfp4::kErrTimeout) ? NVFP4_ERR_TIMEOUT : NVFP4_OK;
+}
+
+nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream_) {
+    if (timeout_ns < 1000ull || timeout_ns > 5000000000ull) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    nvfp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>(timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // extern "C"

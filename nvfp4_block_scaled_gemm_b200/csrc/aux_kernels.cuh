@@ -1,0 +1,150 @@
+// Quantize-and-pack, scale re-layout and the wait-timeout diagnostic kernel.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+// ------------------------------------------------------------ scale re-layout
+// Row-major E4M3 scales [rows][K/16] -> 512-byte atoms (128 rows x 4 blocks):
+// row r, block j of an atom at byte 16*(r%32) + 4*(r/32) + j; atoms ordered
+// along K (one per 64-element MMA step) within each 128-row block; padding
+// rows are zero.  One thread writes one 16-byte line of an atom: the word of
+// K step `ks` from rows L, L+32, L+64, L+96 of row block `rb`.
+__global__ void swizzle_scales_kernel(const uint8_t* __restrict__ s, int rows, int kb_row, int steps,
+                                      long long lines, uint8_t* __restrict__ out) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= lines) return;
+    const int L = (int)(idx & 31);
+    const long long t = idx >> 5;
+    const int ks = (int)(t % steps);
+    const long long rb = t / steps;
+    uint32_t w[4];
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+        const long long r = rb * 128 + L + 32 * r1;
+        w[r1] = r < rows ? __ldg(reinterpret_cast<const uint32_t*>(s + r * kb_row + 4 * ks)) : 0u;
+    }
+    *reinterpret_cast<uint4*>(out + (rb * steps + ks) * 512 + 16 * L) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ------------------------------------------------------------ quantization
+// Pass 1: amax over the tensor, as the bit pattern of a non-negative float
+// (monotone as an unsigned integer) accumulated with atomicMax.
+__global__ void amax_kernel(const float4* __restrict__ x, long long n4, unsigned* __restrict__ amax_bits) {
+    float m = 0.0f;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+        const float4 v = __ldg(x + i);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float warp_max[32];
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(m));
+    }
+}
+
+__device__ __forceinline__ float global_scale_from_amax(float amax) {
+    return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);   // 6 * 448
+}
+
+// Non-negative float -> E4M3, round to nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_from_float(float t) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+    return r & 0xFFu;
+}
+
+// E4M3 byte (sign bit clear) -> its exact float value.
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+    const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+    if (e == 0) return (float)m * 0.001953125f;                 // m * 2^-9
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));     // (1 + m/8) 2^(e-7)
+}
+
+// Eight fp32 values -> eight E2M1 codes (RNE, saturating at 6), element 2i in
+// the low nibble of byte i.  A code whose magnitude rounds to zero carries the
+// sign of its input.
+__device__ __forceinline__ uint32_t e2m1x8_from_float(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t nib = (r >> (4 * i)) & 0xFu;
+        const uint32_t fixed = (nib & 7u) ? nib : (__float_as_uint(v[i]) >> 31) << 3;
+        r = (r & ~(0xFu << (4 * i))) | (fixed << (4 * i));
+    }
+    return r;
+}
+
+// Pass 2: one thread per 16-element block.
+__global__ void quantize_kernel(const float* __restrict__ X, long long blocks, const unsigned* __restrict__ amax_bits,
+                                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= blocks) return;
+    const float g = global_scale_from_amax(__uint_as_float(*amax_bits));
+    const float six_g = __fmul_rn(6.0f, g);
+    float x[16];
+    const float4* src = reinterpret_cast<const float4*>(X + b * 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 f = __ldg(src + i);
+        x[4 * i] = f.x;
+        x[4 * i + 1] = f.y;
+        x[4 * i + 2] = f.z;
+        x[4 * i + 3] = f.w;
+    }
+    float amax_blk = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax_blk = fmaxf(amax_blk, fabsf(x[i]));
+    const uint32_t s = e4m3_from_float(__fdiv_rn(amax_blk, six_g));
+    const float denom = __fmul_rn(g, e4m3_to_float(s));
+    uint32_t out[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = denom == 0.0f ? x[8 * h + i] * 0.0f : __fdiv_rn(x[8 * h + i], denom);
+        out[h] = e2m1x8_from_float(v);
+    }
+    *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(out[0], out[1]);
+    scales[b] = (uint8_t)s;
+}
+
+// Pass 3: replace the amax bits by the global scale g.
+__global__ void finalize_global_scale_kernel(float* g_inout) {
+    g_inout[0] = global_scale_from_amax(__uint_as_float(*reinterpret_cast<unsigned*>(g_inout)));
+}
+
+// ------------------------------------------------------------ diagnostics
+// Waits on a barrier nothing arrives on, bounded by limit_ns; records the
+// timeout in the error word and returns.
+__global__ void wait_timeout_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(smem_addr(&bar), 0, &abort_flag, limit_ns);
+    __syncthreads();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,208 @@
+"""GPU parity of the CUDA path against the CPU oracle, through the C ABI.
+
+Inputs come from the shared generator and are quantised by the ORACLE; the
+GPU GEMM result must satisfy, element by element,
+    |gpu - ref| <= 2^-8 |ref| + 2^-20 |alpha| sum_k |a_k b_k|
+(ref = the exact value).  The quantiser and the scale re-layout are integer
+work and must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_block_scaled_gemm_b200 import synth
+from tests.helpers import quantized_problem, violations
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_block_scaled_gemm_b200 as nv
+    nv.lib()
+    return nv
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def run_gemm(nv, ca, sa, cb, sb, alpha):
+    D = nv.gemm(dev(ca), dev(sa), dev(cb), dev(sb), alpha)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    return D.float().cpu().numpy()
+
+
+# ------------------------------------------------------------------ quantize
+@pytest.mark.parametrize("rows,K,kind,seed", [
+    (8, 6144, "normal", 1000), (33, 512, "moe", 7), (17, 256, "uniform", 3), (1, 16, "normal", 5),
+    (64, 2048, "moe", 11), (3, 8192, "uniform", 13)])
+def test_quantize_bitexact(nv, rows, K, kind, seed):
+    X = synth.source(kind, rows, 8, K, seed)[0]
+    c, s, g = oracle.quantize(X)
+    gc, gs, gg = nv.quantize(dev(X))
+    torch.cuda.synchronize()
+    assert np.float32(gg.item()) == np.float32(g)
+    assert (gs.cpu().numpy() == s).all()
+    assert (gc.cpu().numpy() == c).all()
+
+
+def test_quantize_rounding_edges_bitexact(nv):
+    # Values placed on E2M1 midpoints, E4M3 midpoints, zeros of both signs,
+    # tiny magnitudes and saturating blocks, to pin the hardware conversions
+    # against the oracle's nearest-even definition.
+    K = 256
+    rng = np.random.default_rng(99)
+    X = np.zeros((6, K), np.float32)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 5.5, 6.0, 0.1], np.float32)
+    X[0, :] = np.resize(np.concatenate([mids, -mids]), K)
+    X[0, ::16] = 6.0                                   # g*s == 1 in every block: exact midpoints
+    X[1, :] = -0.0
+    X[1, 5] = 1e-30
+    X[2, :] = rng.standard_normal(K).astype(np.float32) * np.float32(1e-6)
+    X[2, 0] = 6.0
+    X[3, :] = np.resize(np.array([1.0, -1.0, 0.0, 3e-3], np.float32), K)
+    X[4, :] = rng.uniform(-6, 6, K).astype(np.float32)
+    X[5, :] = rng.standard_normal(K).astype(np.float32) * np.exp(rng.uniform(-12, 3, K)).astype(np.float32)
+    c, s, g = oracle.quantize(X)
+    gc, gs, gg = nv.quantize(dev(X))
+    torch.cuda.synchronize()
+    assert np.float32(gg.item()) == np.float32(g)
+    assert (gs.cpu().numpy() == s).all()
+    assert (gc.cpu().numpy() == c).all()
+
+
+# ------------------------------------------------------------------ swizzle
+@pytest.mark.parametrize("rows,K", [(1, 64), (128, 256), (200, 6144), (257, 512)])
+def test_swizzle_bitexact(nv, rows, K):
+    s = synth.random_scales(rows, K, rows + K)
+    ref = oracle.swizzle_scales(s, rows, K)
+    got = nv.swizzle_scales(dev(s), K)
+    torch.cuda.synchronize()
+    assert (got.cpu().numpy() == ref).all()
+
+
+# ------------------------------------------------------------------ GEMM
+SHAPES = [
+    # (M, N, K, kind, seed): the pages' shapes at small M, plus ragged tails
+    (8, 768, 6144, "normal", 1000),      # single GEMM M=8 (attention projection)
+    (1, 768, 6144, "normal", 1100),
+    (16, 256, 6144, "moe", 1201),
+    (64, 2048, 1024, "moe", 1202),
+    (128, 768, 512, "normal", 1103),
+    (129, 264, 512, "uniform", 21),      # first non-swapped size, ragged tiles
+    (300, 520, 1024, "uniform", 22),
+    (5, 40, 64, "normal", 23),           # one K step
+    (37, 136, 320, "moe", 24),           # K tail: 5 steps = 1 stage + 1 step
+    (256, 256, 2048, "uniform", 25),
+    (512, 768, 768, "normal", 26),
+]
+
+
+@pytest.mark.parametrize("M,N,K,kind,seed", SHAPES)
+def test_gemm_matches_oracle(nv, M, N, K, kind, seed):
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, kind, seed)
+    D, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+    got = run_gemm(nv, ca, sa, cb, sb, alpha)
+    bad = violations(got, ref, ad)
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside the bound; first at {np.argwhere(bad)[:3].tolist()}"
+    # the output is non-zero where the exact value is (the "silently zero" failure)
+    assert np.count_nonzero(got) >= 0.99 * np.count_nonzero(ref)
+
+
+def test_gemm_random_codes_all_scales(nv):
+    # every code value and a wide spread of scales, including E4M3 subnormals
+    M, N, K = 96, 200, 1024
+    ca, cb = synth.random_codes(M, K, 1), synth.random_codes(N, K, 2)
+    sa = synth.random_scales(M, K, 3, lo=0x00, hi=0x7E)
+    sb = synth.random_scales(N, K, 4, lo=0x00, hi=0x7E)
+    alpha = 3.0e-5
+    _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+    got = run_gemm(nv, ca, sa, cb, sb, alpha)
+    assert not violations(got, ref, ad).any()
+
+
+@pytest.mark.parametrize("M", [3, 200])
+def test_gemm_one_hot_pins_layouts(nv, M):
+    # Row m of A is a single 1.0 at k = km[m]: D[m, n] = alpha sA[m, km/16] B[n, km] sB[n, km/16],
+    # which pins the nibble order, the K position of every scale block and the row mapping.
+    N, K = 136, 512
+    rng = np.random.default_rng(M)
+    km = rng.integers(0, K, M)
+    A = np.zeros((M, K // 2), np.uint8)
+    for m, k in enumerate(km):
+        A[m, k // 2] = 0x2 << (4 * (k % 2))
+    sa = synth.random_scales(M, K, 5)
+    cb = synth.random_codes(N, K, 6)
+    sb = synth.random_scales(N, K, 7)
+    _, ref, ad = oracle.gemm(A, sa, cb, sb, 1.0, M, N, K)
+    got = run_gemm(nv, A, sa, cb, sb, 1.0)
+    assert not violations(got, ref, ad).any()
+    assert np.count_nonzero(ref) > 0
+
+
+def test_gemm_alpha_is_applied(nv):
+    ca, sa, cb, sb, alpha = quantized_problem(16, 128, 256, "normal", 31)
+    g1 = run_gemm(nv, ca, sa, cb, sb, 1.0)
+    g2 = run_gemm(nv, ca, sa, cb, sb, 0.5)
+    assert np.abs(g1).max() > 0
+    assert (g2 == (g1 * 0.5)).all()      # scaling by a power of two is exact in bf16 here
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 768, 6144), (256, 768, 6144), (2048, 2048, 512)])
+def test_gemm_deterministic(nv, M, N, K):
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "normal", 41)
+    A, SA, B, SB = dev(ca), dev(sa), dev(cb), dev(sb)
+    d1 = nv.gemm(A, SA, B, SB, alpha).clone()
+    d2 = nv.gemm(A, SA, B, SB, alpha)
+    torch.cuda.synchronize()
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+def test_gemm_does_not_write_outside_D(nv):
+    M, N, K = 37, 136, 320
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "normal", 51)
+    guard = 4096
+    buf = torch.full((M * N + 2 * guard,), 12345.0, dtype=torch.bfloat16, device="cuda")
+    D = buf[guard:guard + M * N].view(M, N)
+    nv.gemm(dev(ca), dev(sa), dev(cb), dev(sb), alpha, out=D)
+    torch.cuda.synchronize()
+    assert (buf[:guard] == 12345.0).all() and (buf[guard + M * N:] == 12345.0).all()
+
+
+def test_shape_mismatch_raises(nv):
+    A = torch.zeros((4, 64), dtype=torch.uint8, device="cuda")      # K = 128
+    B = torch.zeros((8, 128), dtype=torch.uint8, device="cuda")     # K = 256
+    with pytest.raises(ValueError, match="K mismatch"):
+        nv.gemm(A, torch.zeros((4, 8), dtype=torch.uint8, device="cuda"), B,
+                torch.zeros((8, 16), dtype=torch.uint8, device="cuda"), 1.0)
+
+
+# ------------------------------------------------------------------ full-size sampled parity
+FULL = [(m, 768, 6144, "normal", 1100 + i) for i, m in enumerate(synth.ATTN_SWEEP_M)] + [
+    (2048, 2048, 6144, "moe", 1205), (512, 256, 6144, "moe", 1214), (2048, 2048, 6144, "uniform", 1300)]
+
+
+@pytest.mark.parametrize("M,N,K,kind,seed", FULL)
+def test_full_size_sampled(nv, M, N, K, kind, seed):
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, kind, seed)
+    got = run_gemm(nv, ca, sa, cb, sb, alpha)
+    rng = np.random.default_rng(seed)
+    n = 3000
+    rows = np.concatenate([rng.integers(0, M, n), [0, M - 1, M - 1]])
+    cols = np.concatenate([rng.integers(0, N, n), [0, N - 1, 0]])
+    _, ref, ad = oracle.gemm_sampled(ca, sa, cb, sb, alpha, M, N, K, rows, cols)
+    assert not violations(got[rows, cols], ref, ad).any()
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_wait_timeout_reports_and_context_survives(nv):
+    assert nv.get_device_error() == 0
+    nv.debug_wait_timeout(20_000_000)            # 20 ms on a barrier nothing arrives on
+    assert nv.get_device_error() == 5            # NVFP4_ERR_TIMEOUT
+    assert nv.get_device_error() == 0            # cleared
+    ca, sa, cb, sb, alpha = quantized_problem(8, 128, 256, "normal", 61)
+    _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, 8, 128, 256)
+    assert not violations(run_gemm(nv, ca, sa, cb, sb, alpha), ref, ad).any()
