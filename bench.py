@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark: NVFP4 GEMM on the attention-projection M-sweep (N=768, K=6144).
+
+One step = one pass of the hot path over the sweep M in {1,16,64,128,256,512}:
+six NVFP4 GEMMs through the C ABI (row-major scales in, BF16 out), each on its
+own buffers.  Steps rotate over enough distinct buffer sets that the working
+set between two uses of a buffer is more than 4x the L2 cache, so every step
+streams its operands from HBM.  Steps are replayed from CUDA graphs and timed
+with CUDA events on the launching stream; the metric is algorithmic bytes /
+time (GB/s) with bytes = M*K/2 + N*K/2 + (M+N)*K/16 + 2*M*N per GEMM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs the same per-GPU workload (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from nvfp4_block_scaled_gemm_b200 import accounting, synth  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS & HBM GB/s vs B200 roofline, M-sweep on attn/MoE shapes"
+SWEEP_M = synth.ATTN_SWEEP_M
+N, K = synth.ATTN_N, synth.HIDDEN_K
+SEED0 = 1100
+WORKLOAD = "attention-projection NVFP4 GEMM sweep: M in {1,16,64,128,256,512}, N=768, K=6144, BF16 out"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+def step_bytes() -> int:
+    return sum(accounting.gemm_bytes(m, N, K) for m in SWEEP_M)
+
+
+def step_flops() -> int:
+    return sum(accounting.gemm_flops(m, N, K) for m in SWEEP_M)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample_rate(target_s: float, per_gemm_outputs: int | None = None, steps: int = 1):
+    """Time the CPU oracle on a bounded sample of the sweep; return
+    (GB/s-equivalent, seconds, outputs computed, per-GEMM outputs per step).
+
+    The oracle computes sampled outputs one by one (exact dot products of
+    K = 6144); the full-GEMM time is extrapolated as (time per output) x M*N,
+    and the value is the sweep's algorithmic bytes over that extrapolated time.
+    """
+    import oracle  # test infrastructure: only this CPU-baseline leg uses it
+
+    rng = np.random.default_rng(7)
+    problems = []
+    for i, m in enumerate(SWEEP_M):
+        A32, B32 = synth.source("normal", m, N, K, SEED0 + i)
+        ca, sa, ga = oracle.quantize(A32)
+        cb, sb, gb = oracle.quantize(B32)
+        problems.append((m, ca, sa, cb, sb, float(np.float32(ga) * np.float32(gb))))
+    # calibrate: seconds per sampled output
+    t0 = time.perf_counter()
+    for m, ca, sa, cb, sb, al in problems:
+        oracle.gemm_sampled(ca, sa, cb, sb, al, m, N, K, [0] * 4, [0, 1, 2, 3])
+    t_one = (time.perf_counter() - t0) / (4 * len(problems))
+    if per_gemm_outputs is None:
+        per_gemm_outputs = int(max(1, min(4096, target_s / max(t_one, 1e-9) / len(problems) / steps)))
+    t_total, n_out = 0.0, 0
+    full_time = 0.0
+    for _ in range(steps):
+        for m, ca, sa, cb, sb, al in problems:
+            r = rng.integers(0, m, per_gemm_outputs)
+            c = rng.integers(0, N, per_gemm_outputs)
+            t0 = time.perf_counter()
+            oracle.gemm_sampled(ca, sa, cb, sb, al, m, N, K, r, c)
+            dt = time.perf_counter() - t0
+            t_total += dt
+            n_out += per_gemm_outputs
+            full_time += dt / per_gemm_outputs * m * N
+    gbs = step_bytes() * steps / full_time / 1e9
+    return gbs, t_total, n_out, per_gemm_outputs, full_time / steps
+
+
+def cpu_baseline_record(target_s: float = 12.0) -> dict:
+    gbs, secs, n_out, per, t_step = oracle_sample_rate(target_s)
+    return {
+        "value": round(gbs, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": f"{n_out} outputs ({per} per GEMM of the sweep, exact K=6144 dot products, single thread) "
+                  f"in {secs:.1f} s; full-sweep time extrapolated as time/output x M*N = {t_step:.1f} s",
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    REASONS = {
+        0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x1: "gpu_idle",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.period, self.ok = [], period_s, False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self._stop.set()
+        self.t.join()
+        inside = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-3:]
+        reasons = set()
+        for _, _, rs in inside:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([s[1] for s in inside])) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_gemm_b200 as nv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    nv.lib()
+    hbm_gbs, bf16_tf, peak_src = load_peaks()
+
+    # Inputs: seeded fp32 sources quantised on the GPU (not timed).
+    base = []
+    gen = torch.Generator(device=dev)
+    for i, m in enumerate(SWEEP_M):
+        gen.manual_seed(SEED0 + i + 1000 * rank)
+        A32 = torch.randn((m, K), generator=gen, device=dev, dtype=torch.float32)
+        B32 = torch.randn((N, K), generator=gen, device=dev, dtype=torch.float32)
+        ca, sa, ga = nv.quantize(A32)
+        cb, sb, gb = nv.quantize(B32)
+        alpha = float(ga.item() * gb.item())
+        base.append((m, ca, sa, cb, sb, alpha))
+        del A32, B32
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    set_bytes = sum(accounting.gemm_bytes(m, N, K) for m in SWEEP_M)
+    R = max(2, -(-4 * l2 // set_bytes))
+    sets = []
+    for r in range(R):
+        sets.append([(m, ca.clone(), sa.clone(), cb.clone(), sb.clone(), al,
+                      torch.empty((m, N), dtype=torch.bfloat16, device=dev)) for (m, ca, sa, cb, sb, al) in base])
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def enqueue_step(r):
+        for (m, ca, sa, cb, sb, al, D) in sets[r]:
+            nv.gemm(ca, sa, cb, sb, al, out=D, stream=stream)
+
+    # Eager warm-up on the capture stream (allocates the library scratch once).
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            enqueue_step(r)
+    stream.synchronize()
+    assert nv.get_device_error(stream) == 0
+
+    # One graph = R consecutive steps (sets 0..R-1); a remainder graph if needed.
+    def capture(nsteps):
+        g = torch.cuda.CUDAGraph()
+        l0 = nv.kernel_launches()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(nsteps):
+                enqueue_step(r % R)
+        return g, nv.kernel_launches() - l0
+
+    g_full, launches_full = capture(R)
+    rem = args.steps % R
+    g_rem, launches_rem = capture(rem) if rem else (None, 0)
+
+    def run_steps(nsteps):
+        launches = 0
+        for _ in range(nsteps // R):
+            g_full.replay()
+            launches += launches_full
+        if nsteps % R:
+            assert nsteps % R == rem and g_rem is not None
+            g_rem.replay()
+            launches += launches_rem
+        return launches
+
+    # Exactly W untimed warm-up steps: whole-graph replays, then eager steps.
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup // R):
+            g_full.replay()
+        for r in range(args.warmup % R):
+            enqueue_step(r)
+    stream.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        launches = run_steps(args.steps)
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    clock_rec = clocks.stop(t_wall0, t_wall1)
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = nv.get_device_error(stream)
+    if status != 0:
+        raise RuntimeError(f"device error status {status}")
+
+    total_bytes = step_bytes() * args.steps * world
+    total_flops = step_flops() * args.steps * world
+    gbs = total_bytes / (ms / 1e3) / 1e9
+    tflops = total_flops / (ms / 1e3) / 1e12
+
+    # Per-GEMM breakdown: one instrumented replay of R steps with an event pair
+    # around every GEMM (separate from the timed region above).
+    per_m = {m: [] for m in SWEEP_M}
+    evs = []
+    gi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gi, stream=stream):
+        for r in range(R):
+            for (m, ca, sa, cb, sb, al, D) in sets[r]:
+                e_a, e_b = torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(
+                    enable_timing=True, external=True)
+                e_a.record(stream)
+                nv.gemm(ca, sa, cb, sb, al, out=D, stream=stream)
+                e_b.record(stream)
+                evs.append((m, e_a, e_b))
+    with torch.cuda.stream(stream):
+        gi.replay()
+    stream.synchronize()
+    for m, e_a, e_b in evs:
+        per_m[m].append(e_a.elapsed_time(e_b))
+    sweep = []
+    for m in SWEEP_M:
+        us = float(np.mean(per_m[m])) * 1e3
+        b, f = accounting.gemm_bytes(m, N, K), accounting.gemm_flops(m, N, K)
+        sweep.append({"M": m, "us": round(us, 3), "GBps": round(b / us / 1e3, 1), "TFLOPS": round(f / us / 1e6, 2),
+                      "hbm_frac": round(b / us / 1e3 / hbm_gbs, 4)})
+
+    # Roofline of the dominant kernel (the GEMM kernel: every launch in a step
+    # is one GEMM launch).  Average launch duration over the timed region.
+    launches_per_rank = launches
+    avg_launch_us = ms * 1e3 / max(1, launches_per_rank)
+    bytes_per_launch = step_bytes() / len(SWEEP_M)
+    achieved = bytes_per_launch / (avg_launch_us * 1e-6) / 1e9
+    traffic = load_traffic()
+
+    # End-to-end through the public API with host buffers.
+    e2e = run_e2e(nv, torch, dev, base, min(args.steps, 20), stream)
+
+    line = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": list(SWEEP_M), "N": N, "K": K, "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2: {R} rotating buffer sets, {R * set_bytes / 2**20:.0f} MiB "
+                         f"vs L2 {l2 / 2**20:.0f} MiB",
+                   "launch": "CUDA graphs of back-to-back nvfp4_gemm calls",
+                   "inputs": "N(0,1) fp32 quantised to NVFP4 on the GPU (not timed)"},
+        "tflops": round(tflops, 3),
+        "sweep": sweep,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": round(achieved / hbm_gbs, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} hbm_gbs",
+                     "per_launch": {"algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_launch_us, 3)}},
+        "e2e": e2e,
+        "gpu_launches": launches_per_rank,
+        "clocks": clock_rec,
+        "accum": "f32", "out_dtype": "bf16",
+    }
+    return line
+
+
+def load_traffic():
+    """DRAM bytes per GEMM launch of the sweep from the committed ncu summary,
+    or None when the kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "traffic_attn_sweep.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("source_hash") != source_hash():
+            return None
+        return rec["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nvfp4_block_scaled_gemm_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def run_e2e(nv, torch, dev, base, steps, stream):
+    """Same metric through nvfp4_gemm with pinned HOST buffers: every step copies
+    its inputs host->device and the outputs device->host inside the timed region."""
+    host = []
+    for (m, ca, sa, cb, sb, al) in base:
+        host.append((m, ca.cpu().pin_memory(), sa.cpu().pin_memory(), cb.cpu().pin_memory(), sb.cpu().pin_memory(),
+                     al, torch.empty((m, N), dtype=torch.bfloat16).pin_memory()))
+    devbuf = [(torch.empty_like(ca, device=dev), torch.empty_like(sa, device=dev), torch.empty_like(cb, device=dev),
+               torch.empty_like(sb, device=dev), torch.empty((m, N), dtype=torch.bfloat16, device=dev))
+              for (m, ca, sa, cb, sb, al, Dh) in host]
+    h2d = sum(x.numel() for (m, ca, sa, cb, sb, al, Dh) in host for x in (ca, sa, cb, sb))
+    d2h = sum(Dh.numel() * 2 for (m, ca, sa, cb, sb, al, Dh) in host)
+
+    def one_step():
+        for (m, ca, sa, cb, sb, al, Dh), (dA, dsA, dB, dsB, dD) in zip(host, devbuf):
+            dA.copy_(ca, non_blocking=True)
+            dsA.copy_(sa, non_blocking=True)
+            dB.copy_(cb, non_blocking=True)
+            dsB.copy_(sb, non_blocking=True)
+            nv.gemm(dA, dsA, dB, dsB, al, out=dD, stream=stream)
+            Dh.copy_(dD, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one_step()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            one_step()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"value": round(step_bytes() * steps / (ms / 1e3) / 1e9, 3), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: each step is a bounded
+    sample of the sweep (a few exact outputs of each GEMM)."""
+    budget_s = 20.0
+    # size the per-step sample so that the K timed steps take about budget_s
+    import oracle
+    probe = oracle_sample_rate(0.0, per_gemm_outputs=4, steps=1)
+    t_out = probe[1] / probe[2]
+    per = int(max(1, min(4096, budget_s / (t_out * len(SWEEP_M) * max(1, args.steps)))))
+    # W untimed warm-up steps (at most 3: the oracle has no warm-up effects)
+    if args.warmup:
+        oracle_sample_rate(0.0, per_gemm_outputs=per, steps=min(args.warmup, 3))
+    gbs, secs, n_out, per, t_step = oracle_sample_rate(0.0, per_gemm_outputs=per, steps=args.steps)
+    value = round(gbs, 6)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int64-exact/f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": list(SWEEP_M), "N": N, "K": K, "parallelism": "cpu1"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{n_out} sampled outputs ({per} per GEMM per step) in {secs:.1f} s; "
+                                   f"full-sweep time extrapolated per output"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline_record()
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -164,6 +164,10 @@ nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 /* Library version as major*10000 + minor*100 + patch. */
 int nvfp4_version(void);
 
+/* Number of kernels this library has enqueued in this process so far, on all
+ * devices (a launch captured into a CUDA graph counts once, at capture). */
+unsigned long long nvfp4_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

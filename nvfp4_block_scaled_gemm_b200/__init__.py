@@ -31,7 +31,7 @@ STATUS = {
 EXPORTS = (
     "nvfp4_gemm", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
-    "nvfp4_debug_wait_timeout", "nvfp4_version",
+    "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
 )
 
 
@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
                      "nvfp4_get_device_error", "nvfp4_debug_wait_timeout"):
             getattr(L, name).restype = i32
         L.nvfp4_version.restype = i32
+        L.nvfp4_kernel_launches.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -186,6 +187,11 @@ def get_device_error(stream=None) -> int:
 
 def debug_wait_timeout(timeout_ns: int, stream=None) -> None:
     _check(lib().nvfp4_debug_wait_timeout(int(timeout_ns), _stream(stream)), "nvfp4_debug_wait_timeout")
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued (or captured) in this process."""
+    return int(lib().nvfp4_kernel_launches())
 
 
 def version() -> int:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <map>
 #include <mutex>
@@ -21,12 +22,15 @@ using nvfp4::TileConfig;
 
 constexpr int kVersion = 100;  // 0.1.0
 
+// Kernels enqueued (or captured into a graph) by this library, all devices.
+std::atomic<unsigned long long> g_launches{0};
+
 // ------------------------------------------------------------ device checks
 struct DeviceInfo {
     bool checked = false;
     bool supported = false;
     int num_sms = 0;
-    unsigned smem_attr_set = 0;  // bit per kernel instantiation
+    uint64_t smem_attr_set = 0;  // bit per kernel instantiation
 };
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_devices;
@@ -55,10 +59,8 @@ nvfp4_status current_device(int* dev, DeviceInfo** info) {
 }
 
 // ------------------------------------------------------------ scratch
-// Per (device, stream) scratch.  Layout: [split-K tile counters, kCounterBytes,
-// zero between launches][everything else].
-constexpr size_t kCounterBytes = 16384;
-constexpr int kMaxCounters = (int)(kCounterBytes / sizeof(unsigned));
+// Per (device, stream) scratch: the re-laid-out scales when they cannot be
+// loaded row-major by TMA.
 
 struct Scratch {
     uint8_t* ptr = nullptr;
@@ -83,10 +85,6 @@ nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** o
         if (cudaMalloc(&p, want) != cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_NO_MEMORY;
-        }
-        if (cudaMemsetAsync(p, 0, kCounterBytes, stream) != cudaSuccess) {
-            cudaFree(p);
-            return NVFP4_ERR_CUDA;
         }
         s.ptr = static_cast<uint8_t*>(p);
         s.cap = want;
@@ -130,6 +128,20 @@ bool make_operand_map(CUtensorMap* map, const void* base, long long rows, long l
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over row-major scales [rows][row_bytes] (row_bytes a multiple of
+// 16); box 16 bytes (= 256 elements of K) x box_rows, no swizzle.
+bool make_scale_map(CUtensorMap* map, const void* base, long long rows, long long row_bytes, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {16u, (cuuint32_t)box_rows};
+    const cuuint32_t elem_strides[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 nvfp4_status launch_swizzle(const void* s, int rows, int K, void* out, cudaStream_t stream) {
@@ -140,6 +152,7 @@ nvfp4_status launch_swizzle(const void* s, int rows, int K, void* out, cudaStrea
     const long long blocks = (lines + threads - 1) / threads;
     nvfp4::swizzle_scales_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
         static_cast<const uint8_t*>(s), rows, K / 16, steps, lines, static_cast<uint8_t*>(out));
+    g_launches++;
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -148,7 +161,7 @@ struct Plan {
     bool swap;
     int bq;
     int tiles_p, tiles_q;
-    int splits, k_tiles, k_per_split;
+    int splits, k_tiles;   // splits = thread-block cluster size along K
 };
 
 Plan make_plan(int M, int N, int K, int num_sms) {
@@ -165,19 +178,25 @@ Plan make_plan(int M, int N, int K, int num_sms) {
         p.tiles_p = (M + 127) / 128;
         p.tiles_q = (N + p.bq - 1) / p.bq;
     }
+    // Split K over a cluster of up to 8 CTAs (a power of two, so that the
+    // 128 tile rows divide evenly in the reduction) while the grid still
+    // fits in one wave.
     const int tiles = p.tiles_p * p.tiles_q;
     int splits = 1;
-    if (tiles < num_sms && tiles <= kMaxCounters) splits = std::max(1, std::min(p.k_tiles, num_sms / tiles));
-    p.k_per_split = (p.k_tiles + splits - 1) / splits;
-    p.splits = (p.k_tiles + p.k_per_split - 1) / p.k_per_split;
+    while (splits * 2 <= 8 && splits * 2 <= p.k_tiles && tiles * splits * 2 <= num_sms) splits *= 2;
+    p.splits = splits;
     return p;
 }
 
-template <int BQ, bool SWAP, bool SPLITK>
-nvfp4_status launch_gemm_kernel(DeviceInfo* info, unsigned bit, const CUtensorMap& tmP, const CUtensorMap& tmQ,
-                                const GemmParams& prm, dim3 grid, cudaStream_t stream) {
+struct Maps {
+    CUtensorMap p, q, sp, sq;
+};
+
+template <int BQ, bool SWAP, bool SPLITK, bool SFR>
+nvfp4_status launch_gemm_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, const GemmParams& prm, dim3 grid,
+                                cudaStream_t stream) {
     using C = TileConfig<BQ>;
-    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK>;
+    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK, SFR>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!(info->smem_attr_set & bit)) {
@@ -186,22 +205,58 @@ nvfp4_status launch_gemm_kernel(DeviceInfo* info, unsigned bit, const CUtensorMa
             info->smem_attr_set |= bit;
         }
     }
-    kern<<<grid, nvfp4::kThreads, C::SMEM_BYTES, stream>>>(tmP, tmQ, prm);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(nvfp4::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    // Let this kernel's launch and prologue overlap the previous kernel in
+    // the stream; the kernel waits for it before touching global memory.
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (SPLITK) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = grid.x;   // the split-K CTAs of one tile
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m.p, m.q, m.sp, m.sq, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
 }
 
-template <bool SWAP, bool SPLITK>
-nvfp4_status launch_by_bq(int bq, DeviceInfo* info, const CUtensorMap& tmP, const CUtensorMap& tmQ,
-                          const GemmParams& prm, dim3 grid, cudaStream_t stream) {
-    const unsigned base = (SWAP ? 1u : 0u) * 10u + (SPLITK ? 5u : 0u);
+template <bool SWAP, bool SPLITK, bool SFR>
+nvfp4_status launch_by_bq(int bq, DeviceInfo* info, const Maps& m, const GemmParams& prm, dim3 grid,
+                          cudaStream_t stream) {
+    const int base = (SWAP ? 1 : 0) * 20 + (SPLITK ? 10 : 0) + (SFR ? 5 : 0);
     switch (bq) {
-        case 16: return launch_gemm_kernel<16, SWAP, SPLITK>(info, 1u << (base + 0), tmP, tmQ, prm, grid, stream);
-        case 32: return launch_gemm_kernel<32, SWAP, SPLITK>(info, 1u << (base + 1), tmP, tmQ, prm, grid, stream);
-        case 64: return launch_gemm_kernel<64, SWAP, SPLITK>(info, 1u << (base + 2), tmP, tmQ, prm, grid, stream);
-        case 128: return launch_gemm_kernel<128, SWAP, SPLITK>(info, 1u << (base + 3), tmP, tmQ, prm, grid, stream);
-        case 256: return launch_gemm_kernel<256, SWAP, SPLITK>(info, 1u << (base + 4), tmP, tmQ, prm, grid, stream);
+        case 16: return launch_gemm_kernel<16, SWAP, SPLITK, SFR>(info, 1ull << (base + 0), m, prm, grid, stream);
+        case 32: return launch_gemm_kernel<32, SWAP, SPLITK, SFR>(info, 1ull << (base + 1), m, prm, grid, stream);
+        case 64: return launch_gemm_kernel<64, SWAP, SPLITK, SFR>(info, 1ull << (base + 2), m, prm, grid, stream);
+        case 128: return launch_gemm_kernel<128, SWAP, SPLITK, SFR>(info, 1ull << (base + 3), m, prm, grid, stream);
+        case 256: return launch_gemm_kernel<256, SWAP, SPLITK, SFR>(info, 1ull << (base + 4), m, prm, grid, stream);
         default: return NVFP4_ERR_UNSUPPORTED_SHAPE;
     }
+}
+
+template <bool SFR>
+nvfp4_status launch_mode(const Plan& plan, DeviceInfo* info, const Maps& m, const GemmParams& prm, dim3 grid,
+                         cudaStream_t stream) {
+    if (plan.swap)
+        return plan.splits > 1 ? launch_by_bq<true, true, SFR>(plan.bq, info, m, prm, grid, stream)
+                               : launch_by_bq<true, false, SFR>(plan.bq, info, m, prm, grid, stream);
+    return plan.splits > 1 ? launch_by_bq<false, true, SFR>(plan.bq, info, m, prm, grid, stream)
+                           : launch_by_bq<false, false, SFR>(plan.bq, info, m, prm, grid, stream);
 }
 
 nvfp4_status check_gemm_args(const void* A, const void* sA, const void* B, const void* sB, const void* D, int M,
@@ -220,6 +275,8 @@ nvfp4_status check_gemm_args(const void* A, const void* sA, const void* B, const
 extern "C" {
 
 int nvfp4_version(void) { return kVersion; }
+
+unsigned long long nvfp4_kernel_launches(void) { return g_launches.load(); }
 
 const char* nvfp4_status_string(nvfp4_status s) {
     switch (s) {
@@ -275,8 +332,10 @@ nvfp4_status nvfp4_quantize(const float* X, int rows, int K, void* codes, void* 
         nvfp4::quantize_kernel<<<(unsigned)((nb + threads - 1) / threads), threads, 0, stream>>>(
             X, nb, reinterpret_cast<const unsigned*>(g_out), static_cast<uint8_t*>(codes),
             static_cast<uint8_t*>(scales));
+        g_launches += 2;
     }
     nvfp4::finalize_global_scale_kernel<<<1, 1, 0, stream>>>(g_out);
+    g_launches++;
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -298,44 +357,47 @@ nvfp4_status nvfp4_gemm(const void* A, const void* sA, const void* B, const void
     const int rows_p = plan.swap ? N : M;
     const int rows_q = plan.swap ? M : N;
 
-    const size_t sfp_bytes = nvfp4_swizzled_scale_bytes(rows_p, K);
-    const size_t sfq_bytes = nvfp4_swizzled_scale_bytes(rows_q, K);
-    const size_t part_bytes =
-        plan.splits > 1 ? (size_t)plan.splits * plan.tiles_p * plan.tiles_q * 128 * plan.bq * sizeof(float) : 0;
-    const size_t off_sfp = kCounterBytes;
+    // Scales go to the kernel row-major (re-laid out in shared memory) when a
+    // 256-element K tile of scales is a 16-byte aligned TMA box; otherwise
+    // they are re-laid out in global scratch first.
+    const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
+    const size_t sfp_bytes = sfr ? 0 : nvfp4_swizzled_scale_bytes(rows_p, K);
+    const size_t sfq_bytes = sfr ? 0 : nvfp4_swizzled_scale_bytes(rows_q, K);
+    const size_t off_sfp = 0;
     const size_t off_sfq = align_up(off_sfp + sfp_bytes, 256);
-    const size_t off_part = align_up(off_sfq + sfq_bytes, 256);
     uint8_t* ws = nullptr;
-    st = get_scratch(dev, stream, off_part + part_bytes, &ws);
-    if (st != NVFP4_OK) return st;
+    if (!sfr) {
+        st = get_scratch(dev, stream, off_sfq + sfq_bytes, &ws);
+        if (st != NVFP4_OK) return st;
+    }
 
-    if ((st = launch_swizzle(sP, rows_p, K, ws + off_sfp, stream)) != NVFP4_OK) return st;
-    if ((st = launch_swizzle(sQ, rows_q, K, ws + off_sfq, stream)) != NVFP4_OK) return st;
-
-    CUtensorMap tmP, tmQ;
-    if (!make_operand_map(&tmP, P, rows_p, K / 2, 128) || !make_operand_map(&tmQ, Q, rows_q, K / 2, plan.bq))
+    Maps maps;
+    if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq))
         return NVFP4_ERR_CUDA;
+    if (sfr) {
+        if (!make_scale_map(&maps.sp, sP, rows_p, K / 16, 128) || !make_scale_map(&maps.sq, sQ, rows_q, K / 16, plan.bq))
+            return NVFP4_ERR_CUDA;
+    } else {
+        if ((st = launch_swizzle(sP, rows_p, K, ws + off_sfp, stream)) != NVFP4_OK) return st;
+        if ((st = launch_swizzle(sQ, rows_q, K, ws + off_sfq, stream)) != NVFP4_OK) return st;
+        maps.sp = maps.p;
+        maps.sq = maps.q;
+    }
 
     GemmParams prm{};
-    prm.sfp = ws + off_sfp;
-    prm.sfq = ws + off_sfq;
+    prm.sfp = sfr ? nullptr : ws + off_sfp;
+    prm.sfq = sfr ? nullptr : ws + off_sfq;
     prm.D = static_cast<__nv_bfloat16*>(D);
-    prm.partials = reinterpret_cast<float*>(ws + off_part);
-    prm.counters = reinterpret_cast<unsigned*>(ws);
     prm.alpha = alpha;
     prm.rows_p = rows_p;
     prm.rows_q = rows_q;
     prm.K = K;
     prm.ldd = N;
     prm.k_tiles = plan.k_tiles;
-    prm.k_tiles_per_split = plan.k_per_split;
-    const dim3 grid(plan.tiles_q, plan.tiles_p, plan.splits);
-    if (plan.swap) {
-        return plan.splits > 1 ? launch_by_bq<true, true>(plan.bq, info, tmP, tmQ, prm, grid, stream)
-                               : launch_by_bq<true, false>(plan.bq, info, tmP, tmQ, prm, grid, stream);
-    }
-    return plan.splits > 1 ? launch_by_bq<false, true>(plan.bq, info, tmP, tmQ, prm, grid, stream)
-                           : launch_by_bq<false, false>(plan.bq, info, tmP, tmQ, prm, grid, stream);
+    prm.tiles_q = plan.tiles_q;
+    const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
+    return sfr ? launch_mode<true>(plan, info, maps, prm, grid, stream)
+               : launch_mode<false>(plan, info, maps, prm, grid, stream);
 }
 
 nvfp4_status nvfp4_grouped_gemm(const void* A, const void* sA, const void* B, const void* sB, const float* alpha,
@@ -376,6 +438,7 @@ nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream_) {
     nvfp4_status st = current_device(&dev, &info);
     if (st != NVFP4_OK) return st;
     nvfp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>(timeout_ns);
+    g_launches++;
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

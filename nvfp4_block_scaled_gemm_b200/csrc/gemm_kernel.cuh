@@ -12,15 +12,37 @@
 // through the 128-row MMA side, and the epilogue writes the transpose.
 //
 // Warp roles (192 threads):
-//   warp 0      TMA producer: operand tiles (2-D TMA, 128-byte swizzle) and
-//               scale atoms (bulk copies) into a STAGES-deep ring;
-//   warp 1      TMEM allocator and MMA issuer: per stage, copies the scale
-//               atoms into TMEM (tcgen05.cp) and issues four
-//               tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 each);
-//   warps 2..5  epilogue: TMEM -> registers -> alpha, BF16 -> global, or
-//               fp32 partial sums with a last-arriver reduction (split-K).
-// Ring protocol: full[s] (producer arrive + TMA bytes) and empty[s]
-// (tcgen05.commit after the MMAs that read stage s).  Every wait is bounded.
+//   warp 0      TMA producer: per 256-element K tile, the P and Q operand
+//               tiles (2-D TMA, 128-byte swizzle) and their scales into a
+//               STAGES-deep shared-memory ring.  Scales arrive either as
+//               row-major [rows][16 B] tiles (SFR: one 2-D TMA box per
+//               operand) or already in 512-byte atoms (bulk copies).
+//   warp 1      TMEM allocator and MMA issuer: four
+//               tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 each) per K tile.
+//   warps 2..5  scale writers during the main loop, epilogue afterwards.  Warp
+//               w owns TMEM lane quadrant w % 4; per K tile it moves the
+//               scales of both operands from shared memory into one of
+//               kScaleBuffers rotating TMEM scale buffers with tcgen05.st.
+//               The epilogue: TMEM -> registers -> alpha, BF16 -> global.
+//
+// Scale layout the MMA reads from TMEM (the one tcgen05.cp.32x128b.warpx4
+// produces from a 512-byte atom): for one K step of 64 elements (4 scale
+// bytes per row) and 128 rows, row r's 4 bytes sit in lane r % 32 of every
+// lane quadrant, column base + r / 32.  A writer lane L therefore stores, for
+// K step j, the words of rows L, L+32, L+64, L+96 in columns base + 4j + 0..3.
+// Writing them with tcgen05.st from four warps keeps the single MMA-issuing
+// thread free of copy instructions.
+//
+// Split-K: the CTAs that share an output tile form one thread-block cluster
+// (blockIdx.x = cluster rank = K slice).  Each writes its fp32 partial tile
+// to its own shared memory; after a cluster barrier, rank r sums rows
+// [r*128/S, (r+1)*128/S) over the S partials through distributed shared
+// memory, in rank order (deterministic), and stores them.
+//
+// Barriers: full[s] (producer arrive + TMA bytes), empty[s] (MMA commit:
+// stage s may be refilled), sf_ready[b] (4 writer arrivals: scale buffer b
+// holds this K tile), sf_free[b] (MMA commit: buffer b may be rewritten),
+// accum (MMA commit after the last K tile).  Every wait is bounded.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,6 +58,7 @@ constexpr int kStepK = 64;        // K of one tcgen05.mma (mxf4nvf4, dense)
 constexpr int kAtomBytes = 512;   // scale atom: 128 rows x 4 blocks of 16
 constexpr int kThreads = 192;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
+constexpr int kScaleBuffers = 4;    // rotating TMEM scale buffers
 
 template <int BQ>
 struct TileConfig {
@@ -49,28 +72,28 @@ struct TileConfig {
     static constexpr int STAGES_FIT = (kSmemLimit - 2048) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
-    // TMEM columns: fp32 accumulator [0, BQ), then the scale columns.
-    static constexpr int SFP_COL = BQ < 32 ? 32 : BQ;
-    static constexpr int SFQ_COL = SFP_COL + 16;                       // 4 steps x 4 columns
-    static constexpr int COLS_USED = SFQ_COL + 16 * Q_BLOCKS;
+    // TMEM columns: fp32 accumulator [0, BQ), then kScaleBuffers scale buffers
+    // of (P: 4 steps x 4) + (Q: 4 steps x 4 x Q_BLOCKS) columns.
+    static constexpr int SF_BASE = BQ < 32 ? 32 : BQ;
+    static constexpr int SF_STRIDE = 16 + 16 * Q_BLOCKS;
+    static constexpr int COLS_USED = SF_BASE + kScaleBuffers * SF_STRIDE;
     static constexpr int TMEM_COLS = COLS_USED <= 32 ? 32 : COLS_USED <= 64 ? 64 : COLS_USED <= 128 ? 128
                                    : COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "TMEM columns");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
     static_assert(STAGES >= 2, "stages");
 };
 
 struct GemmParams {
-    const uint8_t* sfp;       // P scales, tensor-core atom layout
-    const uint8_t* sfq;       // Q scales, tensor-core atom layout
+    const uint8_t* sfp;       // P scales, atom layout (non-SFR)
+    const uint8_t* sfq;       // Q scales, atom layout (non-SFR)
     __nv_bfloat16* D;
-    float* partials;          // split-K: [splits][tilesP][tilesQ][128][BQ]
-    unsigned* counters;       // split-K: [tilesP][tilesQ], zero between launches
     float alpha;
     int rows_p, rows_q;       // valid rows of P and Q
     int K;                    // elements, multiple of 64
     int ldd;                  // row stride of D in elements (= N)
     int k_tiles;              // ceil(K / 256)
-    int k_tiles_per_split;
+    int tiles_q;              // tiles along Q; blockIdx.y = tq + tiles_q * tp
 };
 
 template <int BQ, bool SWAP>
@@ -101,30 +124,123 @@ __device__ __forceinline__ void store_tile_chunk(const GemmParams& prm, const fl
     }
 }
 
-template <int BQ, bool SWAP, bool SPLITK>
+// The 16 scale words of one 128-row block for one K tile, in TMEM column
+// order: out[4*j + r1] = scales of row L + 32*r1 for K step j.  SFR: the
+// block is row-major (row r at byte 16*r, word j = step j); otherwise it is
+// four atoms (atom j at byte 512*j, line L holds rows L, L+32, L+64, L+96).
+template <bool SFR>
+__device__ __forceinline__ void gather_scale_words(uint32_t base, int lane, uint32_t (&out)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = ld_shared_v4(SFR ? base + 16u * (lane + 32 * i) : base + 512u * i + 16u * lane);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            // SFR: i = row group r1, k = step j;  atoms: i = step j, k = row group r1
+            const int j = SFR ? k : i, r1 = SFR ? i : k;
+            out[4 * j + r1] = w[k];
+        }
+    }
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank_addr(uint32_t smem_addr_local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr_local), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// Row stride (floats) of a partial tile in shared memory; the +4 keeps the
+// 16-byte accesses of a warp (one row per lane) free of bank conflicts.
+template <int BQ>
+constexpr int kPartLd = BQ + 4;
+
+// Split-K reduction, run by the 128 epilogue threads of cluster rank r:
+// rows [r*128/S, (r+1)*128/S) of the tile, summed over the S partial tiles in
+// rank order, scaled by alpha and stored.
+template <int BQ, bool SWAP>
+__device__ __forceinline__ void reduce_split_rows(const GemmParams& prm, uint32_t part_base, int tp, int q_row0,
+                                                  int t) {
+    const int S = (int)gridDim.x, rank = (int)blockIdx.x;
+    const int rows_per = kBM / S;
+    const int row0 = rank * rows_per;
+    constexpr int C4 = BQ / 4;                     // float4 columns per row
+    const int n4 = rows_per * C4;
+    for (int i = t; i < n4; i += 128) {
+        // swapped: consecutive threads take consecutive P rows (contiguous in D)
+        const int r = SWAP ? (i % rows_per) : (i / C4);
+        const int c4 = SWAP ? (i / rows_per) : (i % C4);
+        const uint32_t off = part_base + (uint32_t)((row0 + r) * kPartLd<BQ> + 4 * c4) * 4u;
+        float4 v[8];
+#pragma unroll
+        for (int z = 0; z < 8; ++z)            // issue every load first ...
+            if (z < S) v[z] = ld_cluster_f4(cluster_rank_addr(off, (uint32_t)z));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int z = 0; z < 8; ++z) {          // ... then add in rank order
+            if (z < S) {
+                acc.x += v[z].x;
+                acc.y += v[z].y;
+                acc.z += v[z].z;
+                acc.w += v[z].w;
+            }
+        }
+        const int p = tp * kBM + row0 + r;
+        const int q = q_row0 + 4 * c4;
+        if (p >= prm.rows_p) continue;
+        const float o[4] = {acc.x * prm.alpha, acc.y * prm.alpha, acc.z * prm.alpha, acc.w * prm.alpha};
+        if (!SWAP) {
+            if (q < prm.rows_q)   // rows_q (= N) is a multiple of 8
+                *reinterpret_cast<uint2*>(prm.D + (size_t)p * prm.ldd + q) =
+                    make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (q + j < prm.rows_q) prm.D[(size_t)(q + j) * prm.ldd + p] = __float2bfloat16_rn(o[j]);
+        }
+    }
+}
+
+template <int BQ, bool SWAP, bool SPLITK, bool SFR>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                       const GemmParams prm) {
     using C = TileConfig<BQ>;
     constexpr int S = C::STAGES;
+    constexpr int NB = kScaleBuffers;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-    // bars[0..S) full, bars[S..2S) empty, bars[2S] accumulator ready
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 1);
+    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB,2S+2NB) sf_free, [2S+2NB] accum
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tq = blockIdx.x, tp = blockIdx.y, split = blockIdx.z;
-    const int kt_begin = split * prm.k_tiles_per_split;
-    const int kt_end = min(prm.k_tiles, kt_begin + prm.k_tiles_per_split);
+    const int split = blockIdx.x, splits = gridDim.x;
+    const int tq = blockIdx.y % prm.tiles_q, tp = blockIdx.y / prm.tiles_q;
+    // even K partition: every slice non-empty while splits <= k_tiles
+    const int kt_begin = (int)((long long)split * prm.k_tiles / splits);
+    const int kt_end = (int)((long long)(split + 1) * prm.k_tiles / splits);
     const int steps_total = prm.K / kStepK;
     const uint32_t smem_base = smem_addr(smem);
     const uint32_t bar_base = smem_addr(bars);
     auto full_bar = [&](int s) { return bar_base + 8u * s; };
     auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
-    const uint32_t accum_bar = bar_base + 8u * (2 * S);
+    auto sf_ready_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
+    auto sf_free_bar = [&](int b) { return bar_base + 8u * (2 * S + NB + b); };
+    const uint32_t accum_bar = bar_base + 8u * (2 * S + 2 * NB);
 
     // Q scale blocks that exist in the (row-padded) atom buffer for this tile.
     const int q_row0 = tq * BQ;
@@ -138,24 +254,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(sf_ready_bar(b), 4);
+            mbar_init(sf_free_bar(b), 1);
+        }
         mbar_init(accum_bar, 1);
         *abort_flag = 0;
-        *last_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
+    if (threadIdx.x == 32) {
+        prefetch_tensor_map(&tmP);
+        prefetch_tensor_map(&tmQ);
+        if (SFR) {
+            prefetch_tensor_map(&tmSP);
+            prefetch_tensor_map(&tmSQ);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above overlaps the previous kernel's tail when launched with
+    // programmatic stream serialisation; global memory is touched only below.
+    grid_launch_dependents();
+    grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tensor_map(&tmP);
-            prefetch_tensor_map(&tmQ);
             // The 128-row side is read by exactly one tile column in the
             // swapped layout (the weights): stream it; keep the shared side.
             const uint64_t pol_p = SWAP ? policy_evict_first() : policy_evict_last();
@@ -165,18 +294,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = it % S;
                 const uint32_t ph = (uint32_t)(it / S) & 1u;
                 if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
-                const int steps = min(4, steps_total - 4 * kt);
-                const uint32_t sf_bytes = (uint32_t)steps * kAtomBytes;
-                mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + C::Q_BYTES + sf_bytes * (1 + q_blocks));
                 const uint32_t st = smem_base + s * C::STAGE_BYTES;
-                tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
-                tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
-                bulk_load(st + C::P_BYTES + C::Q_BYTES,
-                          prm.sfp + ((size_t)tp * steps_total + 4 * kt) * kAtomBytes, sf_bytes, full_bar(s));
-                for (int b = 0; b < q_blocks; ++b) {
-                    bulk_load(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + b * 4 * kAtomBytes,
-                              prm.sfq + ((size_t)(q_block0 + b) * steps_total + 4 * kt) * kAtomBytes, sf_bytes,
-                              full_bar(s));
+                if (SFR) {
+                    // row-major scale tiles: 16 bytes (= 4 K steps) per row
+                    mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + C::Q_BYTES + 16 * kBM + 16 * BQ);
+                    tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
+                    tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
+                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
+                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(s), kt * 16, q_row0,
+                                pol_q);
+                } else {
+                    const int steps = min(4, steps_total - 4 * kt);
+                    const uint32_t sf_bytes = (uint32_t)steps * kAtomBytes;
+                    mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + C::Q_BYTES + sf_bytes * (1 + q_blocks));
+                    tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
+                    tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
+                    bulk_load(st + C::P_BYTES + C::Q_BYTES,
+                              prm.sfp + ((size_t)tp * steps_total + 4 * kt) * kAtomBytes, sf_bytes, full_bar(s));
+                    for (int b = 0; b < q_blocks; ++b) {
+                        bulk_load(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + b * 4 * kAtomBytes,
+                                  prm.sfq + ((size_t)(q_block0 + b) * steps_total + 4 * kt) * kAtomBytes, sf_bytes,
+                                  full_bar(s));
+                    }
                 }
             }
         }
@@ -186,25 +325,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
                 const int s = it % S;
-                const uint32_t ph = (uint32_t)(it / S) & 1u;
-                if (!mbar_wait(full_bar(s), ph, abort_flag)) break;
+                const int b = it % NB;
+                // sf_ready[b] is arrived after the writers saw full[s]: the
+                // operand tiles of stage s have landed as well.
+                if (!mbar_wait(sf_ready_bar(b), (uint32_t)(it / NB) & 1u, abort_flag)) break;
                 tc_fence_after();
                 const int steps = min(4, steps_total - 4 * kt);
                 const uint32_t st = smem_base + s * C::STAGE_BYTES;
-                const uint32_t sfp_s = st + C::P_BYTES + C::Q_BYTES;
-                const uint32_t sfq_s = sfp_s + C::SFP_BYTES;
-                for (int j = 0; j < steps; ++j) {
-                    tc_copy_32x128b_x4(tmem + C::SFP_COL + 4 * j, desc_scale_atom(sfp_s + j * kAtomBytes));
-                    for (int b = 0; b < q_blocks; ++b)
-                        tc_copy_32x128b_x4(tmem + C::SFQ_COL + 4 * C::Q_BLOCKS * j + 4 * b,
-                                           desc_scale_atom(sfq_s + b * 4 * kAtomBytes + j * kAtomBytes));
-                }
+                const uint32_t sf = tmem + C::SF_BASE + b * C::SF_STRIDE;
                 for (int j = 0; j < steps; ++j) {
                     tc_mma_nvf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
-                                idesc, tmem + C::SFP_COL + 4 * j, tmem + C::SFQ_COL + 4 * C::Q_BLOCKS * j,
-                                (it > 0 || j > 0) ? 1u : 0u);
+                                idesc, sf + 4 * j, sf + 16 + 4 * C::Q_BLOCKS * j, (it > 0 || j > 0) ? 1u : 0u);
                 }
                 tc_commit(empty_bar(s));
+                tc_commit(sf_free_bar(b));
             }
             // Always signal the epilogue (also after an abort), and only once
             // every MMA issued above has completed.
@@ -212,77 +346,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // Epilogue: warp w reads TMEM lane quadrant w % 4.
-        const int quad = warp & 3;
-        const int row = quad * 32 + lane;       // row of P within the tile
+        const int quad = warp & 3;               // TMEM lane quadrant of this warp
+        const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+        // ---- scale writers: shared memory -> TMEM scale buffer, per K tile
+        {
+            int it = 0;
+            for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
+                const int s = it % S;
+                const int b = it % NB;
+                const int use = it / NB;
+                int got = 1;
+                if (lane == 0) {
+                    got = mbar_wait(full_bar(s), (uint32_t)(it / S) & 1u, abort_flag) &&
+                          (use == 0 || mbar_wait(sf_free_bar(b), (uint32_t)(use - 1) & 1u, abort_flag));
+                }
+                if (!__shfl_sync(0xffffffffu, got, 0)) break;
+                const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                const uint32_t sf = t_quad + C::SF_BASE + b * C::SF_STRIDE;
+                uint32_t wp[16];
+                gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES, lane, wp);
+                tmem_store_16(sf, wp);
+                if (C::Q_BLOCKS == 1) {
+                    uint32_t wq[16];
+                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq);
+                    tmem_store_16(sf + 16, wq);
+                } else {
+                    // two 128-row blocks: step j uses columns 8j + 4*block + r1
+                    uint32_t wq0[16], wq1[16], wq[32];
+                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq0);
+                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + 4 * kAtomBytes, lane, wq1);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int r1 = 0; r1 < 4; ++r1) {
+                            wq[8 * j + r1] = wq0[4 * j + r1];
+                            wq[8 * j + 4 + r1] = wq1[4 * j + r1];
+                        }
+                    tmem_store_32(sf + 16, wq);
+                }
+                tmem_wait_store();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sf_ready_bar(b));
+            }
+        }
+
+        // ---- epilogue
+        const int row = quad * 32 + lane;        // row of P within the tile
         const int p = tp * kBM + row;
         int ok = 1;
         if (lane == 0) ok = mbar_wait(accum_bar, 0, abort_flag) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         tc_fence_after();
         if (ok && !*abort_flag) {
-            const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16);
-            if (!SPLITK) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < BQ; c0 += 16) {
-                    uint32_t r[16];
-                    tmem_load_16(t_row + c0, r);
-                    tmem_wait_load();
+            for (int c0 = 0; c0 < BQ; c0 += 16) {
+                uint32_t r[16];
+                tmem_load_16(t_quad + c0, r);
+                tmem_wait_load();
+                if (!SPLITK) {
                     float v[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]) * prm.alpha;
                     store_tile_chunk<BQ, SWAP>(prm, v, p, q_row0 + c0);
-                }
-            } else {
-                const int tilesP = gridDim.y, tilesQ = gridDim.x, splits = gridDim.z;
-                const size_t tile_elems = (size_t)kBM * BQ;
-                const size_t tile_id = (size_t)tp * tilesQ + tq;
-                float* mine = prm.partials + ((size_t)split * tilesP * tilesQ + tile_id) * tile_elems + (size_t)row * BQ;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BQ; c0 += 16) {
-                    uint32_t r[16];
-                    tmem_load_16(t_row + c0, r);
-                    tmem_wait_load();
+                } else {
+                    // fp32 partial row into this CTA's shared memory (the ring is idle now)
+                    const uint32_t dst = smem_base + (uint32_t)(row * kPartLd<BQ> + c0) * 4u;
 #pragma unroll
                     for (int c = 0; c < 16; c += 4)
-                        *reinterpret_cast<uint4*>(mine + c0 + c) = make_uint4(r[c], r[c + 1], r[c + 2], r[c + 3]);
-                }
-                __threadfence();
-                named_barrier(1, 128);
-                if (warp == 2 && lane == 0) {
-                    const unsigned prev = atomicAdd(prm.counters + tile_id, 1u);
-                    const int last = (prev == (unsigned)(splits - 1));
-                    if (last) prm.counters[tile_id] = 0;   // ready for the next launch
-                    *last_flag = last;
-                }
-                named_barrier(1, 128);
-                if (*last_flag) {
-                    __threadfence();
-                    const float* base = prm.partials + tile_id * tile_elems + (size_t)row * BQ;
-                    const size_t split_stride = (size_t)tilesP * tilesQ * tile_elems;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < BQ; c0 += 16) {
-                        float v[16];
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) v[c] = 0.0f;
-                        for (int z = 0; z < splits; ++z) {   // fixed order: deterministic
-                            const float4* src = reinterpret_cast<const float4*>(base + z * split_stride + c0);
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const float4 f = __ldcg(src + c);
-                                v[4 * c + 0] += f.x;
-                                v[4 * c + 1] += f.y;
-                                v[4 * c + 2] += f.z;
-                                v[4 * c + 3] += f.w;
-                            }
-                        }
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) v[c] *= prm.alpha;
-                        store_tile_chunk<BQ, SWAP>(prm, v, p, q_row0 + c0);
-                    }
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 4u * c), "r"(r[c]),
+                                     "r"(r[c + 1]), "r"(r[c + 2]), "r"(r[c + 3])
+                                     : "memory");
                 }
             }
         }
+    }
+
+    if (SPLITK) {
+        cluster_sync();   // every partial tile of the cluster is in shared memory
+        if (warp >= 2 && !*abort_flag) reduce_split_rows<BQ, SWAP>(prm, smem_base, tp, q_row0, threadIdx.x - 64);
+        cluster_sync();   // no CTA leaves while a peer still reads its shared memory
     }
 
     tc_fence_before();
