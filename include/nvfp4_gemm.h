@@ -86,6 +86,22 @@ nvfp4_status nvfp4_gemm(const void* A, const void* sA,
                         int M, int N, int K, void* stream);
 
 /*
+ * nvfp4_gemm_ex -- nvfp4_gemm with flags (0 gives exactly nvfp4_gemm).
+ *   NVFP4_GEMM_B_CONSTANT: the caller guarantees that B and sB are not written
+ *   by any work enqueued earlier on `stream` that may still be running (model
+ *   weights).  The kernel then starts loading B before the previous kernel
+ *   on the stream has finished (it still waits for it before reading A or sA
+ *   and before writing D), which hides the memory latency of back-to-back
+ *   weight-streaming GEMMs.  A, sA and D get no such relaxation.
+ *   Other bits: NVFP4_ERR_INVALID_ARG.
+ */
+#define NVFP4_GEMM_B_CONSTANT 1u
+nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA,
+                           const void* B, const void* sB,
+                           float alpha, void* D,
+                           int M, int N, int K, unsigned flags, void* stream);
+
+/*
  * nvfp4_grouped_gemm -- MoE-style grouped GEMM: G independent problems that
  * share N and K.  Rows [row_offsets[g], row_offsets[g+1]) of A are multiplied
  * by B[g] and scaled by alpha[g]:
@@ -97,7 +113,9 @@ nvfp4_status nvfp4_gemm(const void* A, const void* sA,
  *   (this is not checked on the device; violating it is undefined).
  *   D [M_total][N] bf16 (device).
  *   Groups with no rows cost nothing and their B is never read.
- *   Same requirements as nvfp4_gemm, and G >= 1.
+ *   Requirements: as nvfp4_gemm, and G >= 1, K % 256 == 0, sA and sB 16-byte
+ *   aligned (the kernel loads 256-element K tiles of row-major scales with
+ *   TMA); otherwise NVFP4_ERR_UNSUPPORTED_SHAPE / NVFP4_ERR_INVALID_ARG.
  * Sources: MoE routing gives each expert about 16 rows ("Peeling the Kernel
  * Onion", section "The Critical Connection to Real Inference"); persistent
  * grouped GEMM kernels amortise small per-expert problems (same page, section

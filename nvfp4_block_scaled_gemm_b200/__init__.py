@@ -29,7 +29,7 @@ STATUS = {
 
 # Every symbol include/nvfp4_gemm.h declares.
 EXPORTS = (
-    "nvfp4_gemm", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
+    "nvfp4_gemm", "nvfp4_gemm_ex", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
 )
@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.nvfp4_gemm.argtypes = [P, P, P, P, f32, P, i32, i32, i32, P]
+        L.nvfp4_gemm_ex.argtypes = [P, P, P, P, f32, P, i32, i32, i32, ctypes.c_uint, P]
         L.nvfp4_grouped_gemm.argtypes = [P, P, P, P, P, P, i32, P, i32, i32, i32, P]
         L.nvfp4_quantize.argtypes = [P, i32, i32, P, P, P, P]
         L.nvfp4_swizzle_scales.argtypes = [P, i32, i32, P, P]
@@ -62,7 +63,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_status_string.argtypes = [i32]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         L.nvfp4_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
-        for name in ("nvfp4_gemm", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
+        for name in ("nvfp4_gemm", "nvfp4_gemm_ex", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
                      "nvfp4_get_device_error", "nvfp4_debug_wait_timeout"):
             getattr(L, name).restype = i32
         L.nvfp4_version.restype = i32
@@ -99,13 +100,18 @@ def packed_k(a: torch.Tensor) -> int:
     return a.shape[-1] * 2
 
 
+B_CONSTANT = 1
+
+
 def gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, alpha: float,
-         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+         out: torch.Tensor | None = None, stream=None, b_constant: bool = False) -> torch.Tensor:
     """D[M,N] (bf16) = alpha * (A * sA) @ (B * sB)^T.
 
     A uint8 [M, K/2], sA uint8 [M, K/16], B uint8 [N, K/2], sB uint8 [N, K/16].
     K is given by the packed operands: both must hold K/2 bytes per row
     (a mismatch is reported here rather than as a kernel error).
+    b_constant: B and sB are not written by earlier work still running on the
+    stream (weights); lets the kernel start loading them early.
     """
     if A.dim() != 2 or B.dim() != 2:
         raise ValueError("A and B must be 2-D packed E2M1 tensors [rows, K/2]")
@@ -120,8 +126,12 @@ def gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, a
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     _need(out, "out", torch.bfloat16, (M, N))
-    _check(lib().nvfp4_gemm(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
-                            out.data_ptr(), M, N, K, _stream(stream)), "nvfp4_gemm")
+    if b_constant:
+        _check(lib().nvfp4_gemm_ex(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
+                                   out.data_ptr(), M, N, K, B_CONSTANT, _stream(stream)), "nvfp4_gemm_ex")
+    else:
+        _check(lib().nvfp4_gemm(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
+                                out.data_ptr(), M, N, K, _stream(stream)), "nvfp4_gemm")
     return out
 
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <atomic>
 #include <cstdint>
 #include <map>
@@ -14,6 +16,7 @@
 #include "../../include/nvfp4_gemm.h"
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
+#include "grouped_kernel.cuh"
 
 namespace {
 
@@ -164,26 +167,62 @@ struct Plan {
     int splits, k_tiles;   // splits = thread-block cluster size along K
 };
 
-Plan make_plan(int M, int N, int K, int num_sms) {
+// Tuning override: NVFP4_GEMM_PLAN="swap:bq:splits" (e.g. "1:16:8") forces the
+// tile shape of every nvfp4_gemm call whose shape allows it.  Read on each
+// call (a getenv), so a tuning run can change it between calls.
+struct PlanOverride {
+    bool set = false;
+    int swap = 0, bq = 0, splits = 0;
+};
+
+PlanOverride plan_override() {
+    PlanOverride o;
+    const char* e = std::getenv("NVFP4_GEMM_PLAN");
+    int a, b, c;
+    if (e && std::sscanf(e, "%d:%d:%d", &a, &b, &c) == 3 && (b == 16 || b == 32 || b == 64 || b == 128 || b == 256) &&
+        (c == 1 || c == 2 || c == 4 || c == 8)) {
+        o.set = true;
+        o.swap = a != 0;
+        o.bq = b;
+        o.splits = c;
+    }
+    return o;
+}
+
+Plan make_plan(int M, int N, int K, int num_sms, bool sfr) {
     Plan p{};
     p.k_tiles = (K + 255) / 256;
-    if (M <= 128) {
+    const PlanOverride o = plan_override();
+    if (o.set && o.splits <= p.k_tiles) {
+        p.swap = o.swap;
+        p.bq = o.bq;
+        p.tiles_p = o.swap ? (N + 127) / 128 : (M + 127) / 128;
+        p.tiles_q = o.swap ? (M + o.bq - 1) / o.bq : (N + o.bq - 1) / o.bq;
+        p.splits = o.splits;
+        // without row-major scale tiles, a narrow Q tile must start on a 128-row block
+        if (sfr || p.bq >= 128 || p.tiles_q == 1) return p;
+    }
+    // Tile shape (measured on the attention and MoE decode shapes): weight
+    // rows on the 128-row MMA side with narrow token tiles for small M, then
+    // 64- and 128-wide N tiles; 256-wide tiles once the grid is large.
+    if (M <= 64) {
         p.swap = true;
-        p.bq = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
-        p.tiles_p = (N + 127) / 128;
-        p.tiles_q = 1;
+        p.bq = M <= 16 ? 16 : 32;
+        if (!sfr && M > p.bq) p.bq = 64;   // one Q tile: scale atoms start on row 0
     } else {
         p.swap = false;
-        p.bq = N >= 256 ? 256 : 128;
-        p.tiles_p = (M + 127) / 128;
-        p.tiles_q = (N + p.bq - 1) / p.bq;
+        p.bq = M <= 256 ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
     }
-    // Split K over a cluster of up to 8 CTAs (a power of two, so that the
-    // 128 tile rows divide evenly in the reduction) while the grid still
-    // fits in one wave.
+    p.tiles_p = p.swap ? (N + 127) / 128 : (M + 127) / 128;
+    p.tiles_q = p.swap ? (M + p.bq - 1) / p.bq : (N + p.bq - 1) / p.bq;
+    // Split K over a cluster of up to 8 CTAs (a power of two, so that the 128
+    // tile rows divide evenly in the reduction) while the grid stays at or
+    // below ~128 CTAs, which leaves room for the next kernel's CTAs to start
+    // (programmatic dependent launch) on the remaining SMs.
     const int tiles = p.tiles_p * p.tiles_q;
+    const int cap = std::min(num_sms, 128);
     int splits = 1;
-    while (splits * 2 <= 8 && splits * 2 <= p.k_tiles && tiles * splits * 2 <= num_sms) splits *= 2;
+    while (splits * 2 <= 8 && splits * 2 <= p.k_tiles && tiles * splits * 2 <= cap) splits *= 2;
     p.splits = splits;
     return p;
 }
@@ -341,6 +380,12 @@ nvfp4_status nvfp4_quantize(const float* X, int rows, int K, void* codes, void* 
 
 nvfp4_status nvfp4_gemm(const void* A, const void* sA, const void* B, const void* sB, float alpha, void* D, int M,
                         int N, int K, void* stream_) {
+    return nvfp4_gemm_ex(A, sA, B, sB, alpha, D, M, N, K, 0u, stream_);
+}
+
+nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const void* sB, float alpha, void* D, int M,
+                           int N, int K, unsigned flags, void* stream_) {
+    if (flags & ~NVFP4_GEMM_B_CONSTANT) return NVFP4_ERR_INVALID_ARG;
     nvfp4_status st = check_gemm_args(A, sA, B, sB, D, M, N, K);
     if (st != NVFP4_OK || M == 0 || N == 0) return st;
     int dev;
@@ -349,7 +394,12 @@ nvfp4_status nvfp4_gemm(const void* A, const void* sA, const void* B, const void
     if (st != NVFP4_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
-    const Plan plan = make_plan(M, N, K, info->num_sms);
+    // Scales go to the kernel row-major (TMA tiles, laid out for the tensor
+    // cores inside the kernel) when a 256-element K tile of scales is a
+    // 16-byte aligned TMA box; otherwise they are re-laid out in global
+    // scratch first.
+    const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
+    const Plan plan = make_plan(M, N, K, info->num_sms, sfr);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
     const void* sP = plan.swap ? sB : sA;
@@ -357,10 +407,6 @@ nvfp4_status nvfp4_gemm(const void* A, const void* sA, const void* B, const void
     const int rows_p = plan.swap ? N : M;
     const int rows_q = plan.swap ? M : N;
 
-    // Scales go to the kernel row-major (re-laid out in shared memory) when a
-    // 256-element K tile of scales is a 16-byte aligned TMA box; otherwise
-    // they are re-laid out in global scratch first.
-    const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
     const size_t sfp_bytes = sfr ? 0 : nvfp4_swizzled_scale_bytes(rows_p, K);
     const size_t sfq_bytes = sfr ? 0 : nvfp4_swizzled_scale_bytes(rows_q, K);
     const size_t off_sfp = 0;
@@ -395,6 +441,7 @@ nvfp4_status nvfp4_gemm(const void* A, const void* sA, const void* B, const void
     prm.ldd = N;
     prm.k_tiles = plan.k_tiles;
     prm.tiles_q = plan.tiles_q;
+    prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
     const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
     return sfr ? launch_mode<true>(plan, info, maps, prm, grid, stream)
                : launch_mode<false>(plan, info, maps, prm, grid, stream);
@@ -408,12 +455,57 @@ nvfp4_status nvfp4_grouped_gemm(const void* A, const void* sA, const void* B, co
     if (st != NVFP4_OK) return st;
     if (M_total == 0 || N == 0) return NVFP4_OK;
     if (!alpha || !row_offsets || !aligned(alpha, 4) || !aligned(row_offsets, 4)) return NVFP4_ERR_INVALID_ARG;
+    // The grouped kernel loads row-major scale tiles with TMA.
+    if (K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(sA, 16) || !aligned(sB, 16)) return NVFP4_ERR_INVALID_ARG;
     int dev;
     DeviceInfo* info;
     st = current_device(&dev, &info);
     if (st != NVFP4_OK) return st;
-    (void)stream_;
-    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    using GC = nvfp4::GroupedConfig;
+    CUtensorMap tmB, tmA, tmSB, tmSA;
+    const long long b_rows = (long long)G * N;
+    if (!make_operand_map(&tmB, B, b_rows, K / 2, 128) || !make_operand_map(&tmA, A, M_total, K / 2, 16) ||
+        !make_scale_map(&tmSB, sB, b_rows, K / 16, 128) || !make_scale_map(&tmSA, sA, M_total, K / 16, 16))
+        return NVFP4_ERR_CUDA;
+    nvfp4::GroupedParams prm{};
+    prm.alpha = alpha;
+    prm.offsets = row_offsets;
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.G = G;
+    prm.N = N;
+    prm.K = K;
+    prm.M_total = M_total;
+    prm.tiles_n = (N + 127) / 128;
+    prm.k_tiles = K / 256;
+    auto kern = nvfp4::nvfp4_grouped_kernel;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(info->smem_attr_set & (1ull << 63))) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GC::SMEM_BYTES) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            info->smem_attr_set |= (1ull << 63);
+        }
+    }
+    const long long units = (long long)G * prm.tiles_n;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<long long>(units, info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGroupedThreads, 1, 1);
+    cfg.dynamicSmemBytes = GC::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmB, tmA, tmSB, tmSA, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_get_device_error(void* stream_) {

@@ -34,10 +34,11 @@
 // thread free of copy instructions.
 //
 // Split-K: the CTAs that share an output tile form one thread-block cluster
-// (blockIdx.x = cluster rank = K slice).  Each writes its fp32 partial tile
-// to its own shared memory; after a cluster barrier, rank r sums rows
-// [r*128/S, (r+1)*128/S) over the S partials through distributed shared
-// memory, in rank order (deterministic), and stores them.
+// (blockIdx.x = cluster rank = K slice).  Rank r owns rows [r*128/S,
+// (r+1)*128/S) of the tile.  Every CTA stores each fp32 partial row straight
+// from registers into the owner's shared memory (distributed shared memory,
+// slot = the sender's rank); after one cluster barrier each owner sums its S
+// slots in rank order (deterministic), applies alpha and stores BF16.
 //
 // Barriers: full[s] (producer arrive + TMA bytes), empty[s] (MMA commit:
 // stage s may be refilled), sf_ready[b] (4 writer arrivals: scale buffer b
@@ -94,6 +95,7 @@ struct GemmParams {
     int ldd;                  // row stride of D in elements (= N)
     int k_tiles;              // ceil(K / 256)
     int tiles_q;              // tiles along Q; blockIdx.y = tq + tiles_q * tp
+    int prefetch_b;           // B is constant: fetch its first tiles before waiting on the previous grid
 };
 
 template <int BQ, bool SWAP>
@@ -153,48 +155,39 @@ __device__ __forceinline__ uint32_t cluster_rank_addr(uint32_t smem_addr_local, 
     return r;
 }
 
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr));
-    return v;
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
 }
 
-// Row stride (floats) of a partial tile in shared memory; the +4 keeps the
-// 16-byte accesses of a warp (one row per lane) free of bank conflicts.
+// Row stride (floats) of a partial row slot in shared memory; the +4 keeps
+// the 16-byte accesses of a warp (one row per lane) free of bank conflicts.
 template <int BQ>
 constexpr int kPartLd = BQ + 4;
 
-// Split-K reduction, run by the 128 epilogue threads of cluster rank r:
-// rows [r*128/S, (r+1)*128/S) of the tile, summed over the S partial tiles in
-// rank order, scaled by alpha and stored.
+// Split-K reduction, run by the 128 epilogue threads of the owner (cluster
+// rank r) after the cluster barrier: its rows_per rows, summed over the S
+// slots [z][rows_per][kPartLd] in rank order, scaled by alpha and stored.
 template <int BQ, bool SWAP>
-__device__ __forceinline__ void reduce_split_rows(const GemmParams& prm, uint32_t part_base, int tp, int q_row0,
-                                                  int t) {
+__device__ __forceinline__ void reduce_owned_rows(const GemmParams& prm, uint32_t slots, int tp, int q_row0, int t) {
     const int S = (int)gridDim.x, rank = (int)blockIdx.x;
     const int rows_per = kBM / S;
     const int row0 = rank * rows_per;
     constexpr int C4 = BQ / 4;                     // float4 columns per row
     const int n4 = rows_per * C4;
+    const uint32_t slot_bytes = (uint32_t)(rows_per * kPartLd<BQ>) * 4u;
     for (int i = t; i < n4; i += 128) {
         // swapped: consecutive threads take consecutive P rows (contiguous in D)
         const int r = SWAP ? (i % rows_per) : (i / C4);
         const int c4 = SWAP ? (i / rows_per) : (i % C4);
-        const uint32_t off = part_base + (uint32_t)((row0 + r) * kPartLd<BQ> + 4 * c4) * 4u;
-        float4 v[8];
-#pragma unroll
-        for (int z = 0; z < 8; ++z)            // issue every load first ...
-            if (z < S) v[z] = ld_cluster_f4(cluster_rank_addr(off, (uint32_t)z));
+        const uint32_t off = slots + (uint32_t)(r * kPartLd<BQ> + 4 * c4) * 4u;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int z = 0; z < 8; ++z) {          // ... then add in rank order
-            if (z < S) {
-                acc.x += v[z].x;
-                acc.y += v[z].y;
-                acc.z += v[z].z;
-                acc.w += v[z].w;
-            }
+        for (int z = 0; z < S; ++z) {          // rank order
+            const uint4 v = ld_shared_v4(off + (uint32_t)z * slot_bytes);
+            acc.x += __uint_as_float(v.x);
+            acc.y += __uint_as_float(v.y);
+            acc.z += __uint_as_float(v.z);
+            acc.w += __uint_as_float(v.w);
         }
         const int p = tp * kBM + row0 + r;
         const int q = q_row0 + 4 * c4;
@@ -281,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Everything above overlaps the previous kernel's tail when launched with
     // programmatic stream serialisation; global memory is touched only below.
     grid_launch_dependents();
-    grid_dependency_wait();
+    const bool producer = (warp == 0 && lane == 0);
+    if (!producer) grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -289,12 +283,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             // swapped layout (the weights): stream it; keep the shared side.
             const uint64_t pol_p = SWAP ? policy_evict_first() : policy_evict_last();
             const uint64_t pol_q = SWAP ? policy_evict_last() : policy_evict_first();
+            // With a constant B, its first ring's worth of tiles is requested
+            // before waiting for the previous grid (only B is touched then).
+            int pre = 0;
+            if (SFR && prm.prefetch_b) {
+                pre = min(S, kt_end - kt_begin);
+                for (int i = 0; i < pre; ++i) {
+                    const int kt = kt_begin + i;
+                    const uint32_t st = smem_base + i * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(full_bar(i), C::P_BYTES + C::Q_BYTES + 16 * kBM + 16 * BQ);
+                    if (SWAP) {   // B is P
+                        tma_load_2d(st, &tmP, full_bar(i), kt * kStageKBytes, tp * kBM, pol_p);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(i), kt * 16, tp * kBM, pol_p);
+                    } else {      // B is Q
+                        tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(i), kt * kStageKBytes, q_row0, pol_q);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(i), kt * 16, q_row0,
+                                    pol_q);
+                    }
+                }
+            }
+            grid_dependency_wait();
             int it = 0;
             for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (uint32_t)(it / S) & 1u;
-                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
                 const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                if (it < pre) {   // the other operand of a prefetched stage
+                    if (SWAP) {
+                        tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(s), kt * 16, q_row0,
+                                    pol_q);
+                    } else {
+                        tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
+                    }
+                    continue;
+                }
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
                 if (SFR) {
                     // row-major scale tiles: 16 bytes (= 4 K steps) per row
                     mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + C::Q_BYTES + 16 * kBM + 16 * BQ);
@@ -348,84 +373,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         const int quad = warp & 3;               // TMEM lane quadrant of this warp
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
-        // ---- scale writers: shared memory -> TMEM scale buffer, per K tile
+        // ---- scale writers: shared memory -> TMEM scale buffer, per K tile.
+        // When the next K tile has landed too, both are written before the one
+        // tcgen05.wait::st, halving the store round trips.
         {
             int it = 0;
-            for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
-                const int s = it % S;
-                const int b = it % NB;
-                const int use = it / NB;
-                int got = 1;
+            for (int kt = kt_begin; kt < kt_end;) {
+                int got = 1, cnt = 1;
                 if (lane == 0) {
-                    got = mbar_wait(full_bar(s), (uint32_t)(it / S) & 1u, abort_flag) &&
-                          (use == 0 || mbar_wait(sf_free_bar(b), (uint32_t)(use - 1) & 1u, abort_flag));
+                    const int s0 = it % S, b0 = it % NB, use0 = it / NB;
+                    got = mbar_wait(full_bar(s0), (uint32_t)(it / S) & 1u, abort_flag) &&
+                          (use0 == 0 || mbar_wait(sf_free_bar(b0), (uint32_t)(use0 - 1) & 1u, abort_flag));
+                    if (got && kt + 1 < kt_end) {
+                        const int i1 = it + 1, s1 = i1 % S, b1 = i1 % NB, use1 = i1 / NB;
+                        if (mbar_test(full_bar(s1), (uint32_t)(i1 / S) & 1u) &&
+                            (use1 == 0 || mbar_test(sf_free_bar(b1), (uint32_t)(use1 - 1) & 1u)))
+                            cnt = 2;
+                    }
                 }
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
-                const uint32_t st = smem_base + s * C::STAGE_BYTES;
-                const uint32_t sf = t_quad + C::SF_BASE + b * C::SF_STRIDE;
-                uint32_t wp[16];
-                gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES, lane, wp);
-                tmem_store_16(sf, wp);
-                if (C::Q_BLOCKS == 1) {
-                    uint32_t wq[16];
-                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq);
-                    tmem_store_16(sf + 16, wq);
-                } else {
-                    // two 128-row blocks: step j uses columns 8j + 4*block + r1
-                    uint32_t wq0[16], wq1[16], wq[32];
-                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq0);
-                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + 4 * kAtomBytes, lane, wq1);
+                cnt = __shfl_sync(0xffffffffu, cnt, 0);
+                for (int u = 0; u < cnt; ++u) {
+                    const int iu = it + u;
+                    const uint32_t st = smem_base + (iu % S) * C::STAGE_BYTES;
+                    const uint32_t sf = t_quad + C::SF_BASE + (iu % NB) * C::SF_STRIDE;
+                    uint32_t wp[16];
+                    gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES, lane, wp);
+                    tmem_store_16(sf, wp);
+                    if (C::Q_BLOCKS == 1) {
+                        uint32_t wq[16];
+                        gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq);
+                        tmem_store_16(sf + 16, wq);
+                    } else {
+                        // two 128-row blocks: step j uses columns 8j + 4*block + r1
+                        uint32_t wq0[16], wq1[16], wq[32];
+                        gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq0);
+                        gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + 4 * kAtomBytes, lane,
+                                                wq1);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < 4; ++j)
 #pragma unroll
-                        for (int r1 = 0; r1 < 4; ++r1) {
-                            wq[8 * j + r1] = wq0[4 * j + r1];
-                            wq[8 * j + 4 + r1] = wq1[4 * j + r1];
-                        }
-                    tmem_store_32(sf + 16, wq);
+                            for (int r1 = 0; r1 < 4; ++r1) {
+                                wq[8 * j + r1] = wq0[4 * j + r1];
+                                wq[8 * j + 4 + r1] = wq1[4 * j + r1];
+                            }
+                        tmem_store_32(sf + 16, wq);
+                    }
                 }
                 tmem_wait_store();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(sf_ready_bar(b));
+                if (lane == 0)
+                    for (int u = 0; u < cnt; ++u) mbar_arrive(sf_ready_bar((it + u) % NB));
+                it += cnt;
+                kt += cnt;
             }
         }
 
-        // ---- epilogue
-        const int row = quad * 32 + lane;        // row of P within the tile
-        const int p = tp * kBM + row;
+        // ---- epilogue (direct); the split-K epilogue follows the role branches
         int ok = 1;
         if (lane == 0) ok = mbar_wait(accum_bar, 0, abort_flag) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         tc_fence_after();
-        if (ok && !*abort_flag) {
+        if (!SPLITK && ok && !*abort_flag) {
+            const int p = tp * kBM + quad * 32 + lane;
 #pragma unroll 1
             for (int c0 = 0; c0 < BQ; c0 += 16) {
                 uint32_t r[16];
                 tmem_load_16(t_quad + c0, r);
                 tmem_wait_load();
-                if (!SPLITK) {
-                    float v[16];
+                float v[16];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]) * prm.alpha;
-                    store_tile_chunk<BQ, SWAP>(prm, v, p, q_row0 + c0);
-                } else {
-                    // fp32 partial row into this CTA's shared memory (the ring is idle now)
-                    const uint32_t dst = smem_base + (uint32_t)(row * kPartLd<BQ> + c0) * 4u;
-#pragma unroll
-                    for (int c = 0; c < 16; c += 4)
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 4u * c), "r"(r[c]),
-                                     "r"(r[c + 1]), "r"(r[c + 2]), "r"(r[c + 3])
-                                     : "memory");
-                }
+                for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]) * prm.alpha;
+                store_tile_chunk<BQ, SWAP>(prm, v, p, q_row0 + c0);
             }
         }
     }
 
     if (SPLITK) {
-        cluster_sync();   // every partial tile of the cluster is in shared memory
-        if (warp >= 2 && !*abort_flag) reduce_split_rows<BQ, SWAP>(prm, smem_base, tp, q_row0, threadIdx.x - 64);
-        cluster_sync();   // no CTA leaves while a peer still reads its shared memory
+        // Every CTA of the cluster is past its main loop (its accumulator is
+        // final, its ring idle): rows may now be pushed into peers' rings.
+        cluster_sync();
+        if (warp >= 2 && !*abort_flag) {
+            const int quad = warp & 3;
+            const int row = quad * 32 + lane;
+            const int rows_per = kBM / splits;
+            const uint32_t owner = (uint32_t)(row / rows_per);
+            const uint32_t local =
+                smem_base + (uint32_t)((split * rows_per + row % rows_per) * kPartLd<BQ>) * 4u;
+            const uint32_t dst = cluster_rank_addr(local, owner);
+            const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BQ; c0 += 16) {
+                uint32_t r[16];
+                tmem_load_16(t_quad + c0, r);
+                tmem_wait_load();
+#pragma unroll
+                for (int c = 0; c < 16; c += 4)
+                    st_cluster_v4(dst + 4u * (c0 + c), r[c], r[c + 1], r[c + 2], r[c + 3]);
+            }
+        }
+        cluster_sync();   // every partial row has reached its owner
+        if (warp >= 2 && !*abort_flag) reduce_owned_rows<BQ, SWAP>(prm, smem_base, tp, q_row0, threadIdx.x - 64);
     }
 
     tc_fence_before();

@@ -1,0 +1,279 @@
+// Grouped (MoE) NVFP4 GEMM: G problems sharing N and K.  Rows
+// [off[g], off[g+1]) of A multiply expert g's weights B[g] and are scaled by
+// alpha[g] ("Peeling the Kernel Onion", sections "The Critical Connection to
+// Real Inference" -- about 16 rows per expert -- and "Knowledge Created and
+// Its Impact" -- persistent grouped kernels).
+//
+// Persistent kernel.  A work unit is (expert g, 128-row tile of B[g]); CTA b
+// takes units b, b + gridDim.x, ...  The weights sit on the tensor cores'
+// 128-row M side and the expert's tokens on the N side, in passes of up to 128
+// rows; each pass loads only ceil(rows/16) 16-row boxes of A and runs MMAs
+// with N = that many rows rounded up to 16 (the instruction descriptor is
+// built at run time).  Empty experts cost two loads of row_offsets and never
+// touch their weights.
+//
+// Warp roles (320 threads): warp 0 TMA producer; warp 1 TMEM allocator and
+// MMA issuer; warps 2..5 epilogue (TMEM -> alpha[g] -> BF16 -> D); warps 6..9
+// scale writers (shared memory -> TMEM, one warp per lane quadrant, as in the
+// single GEMM kernel).  The fp32 accumulator is double-buffered in TMEM so the
+// epilogue of one pass overlaps the main loop of the next.
+#pragma once
+
+#include "gemm_kernel.cuh"
+
+namespace nvfp4 {
+
+constexpr int kGroupedThreads = 320;
+constexpr int kGroupedBQ = 128;   // max tokens per pass
+
+struct GroupedParams {
+    const float* alpha;           // [G]
+    const int32_t* offsets;       // [G+1]
+    __nv_bfloat16* D;             // [M_total][N]
+    int G, N, K, M_total;
+    int tiles_n;                  // ceil(N / 128)
+    int k_tiles;                  // K / 256
+};
+
+struct GroupedConfig {
+    static constexpr int BQ = kGroupedBQ;
+    static constexpr int P_BYTES = kBM * kStageKBytes;            // 16 KB of weights per K tile
+    static constexpr int Q_BYTES = BQ * kStageKBytes;             // up to 16 KB of tokens
+    static constexpr int SFP_BYTES = 4 * kAtomBytes;
+    static constexpr int SFQ_BYTES = 4 * kAtomBytes;
+    static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
+    static constexpr int STAGES = (kSmemLimit - 2048) / STAGE_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
+    // TMEM: two accumulators [0,128) and [128,256), then 4 scale buffers of 32.
+    static constexpr int ACC_COLS = BQ;
+    static constexpr int SF_BASE = 2 * BQ;
+    static constexpr int SF_STRIDE = 32;
+    static constexpr int TMEM_COLS = 512;
+    static_assert(SF_BASE + kScaleBuffers * SF_STRIDE <= TMEM_COLS, "TMEM columns");
+    static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
+};
+
+// Walks the (unit, pass) sequence of this CTA; every role advances its own
+// copy in the same order.
+struct JobCursor {
+    int unit, units, stride;
+    int g, nt, r0, rows, pass;
+    const GroupedParams* prm;
+
+    __device__ void init(const GroupedParams& p) {
+        prm = &p;
+        units = p.G * p.tiles_n;
+        stride = (int)gridDim.x;
+        unit = (int)blockIdx.x - stride;
+        pass = 0;
+        rows = 0;
+        advance_unit();
+    }
+    __device__ void advance_unit() {
+        for (unit += stride; unit < units; unit += stride) {
+            g = unit / prm->tiles_n;
+            nt = unit % prm->tiles_n;
+            r0 = __ldg(prm->offsets + g);
+            rows = __ldg(prm->offsets + g + 1) - r0;
+            if (rows > 0) break;          // empty experts: nothing to load
+        }
+        pass = 0;
+    }
+    __device__ bool valid() const { return unit < units; }
+    __device__ int q_row0() const { return r0 + pass * kGroupedBQ; }
+    __device__ int q_rows() const { return min(kGroupedBQ, rows - pass * kGroupedBQ); }
+    __device__ void next() {
+        if ((pass + 1) * kGroupedBQ < rows) ++pass;
+        else advance_unit();
+    }
+};
+
+__global__ void __launch_bounds__(kGroupedThreads, 1)
+    nvfp4_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmSB, const __grid_constant__ CUtensorMap tmSA,
+                         const GroupedParams prm) {
+    using C = GroupedConfig;
+    constexpr int S = C::STAGES;
+    constexpr int NB = kScaleBuffers;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB,2S+2NB) sf_free,
+    //       [2S+2NB, +2) acc_full, [2S+2NB+2, +2) acc_empty
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t smem_base = smem_addr(smem);
+    const uint32_t bar_base = smem_addr(bars);
+    auto full_bar = [&](int s) { return bar_base + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
+    auto sf_ready_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
+    auto sf_free_bar = [&](int b) { return bar_base + 8u * (2 * S + NB + b); };
+    auto acc_full_bar = [&](int a) { return bar_base + 8u * (2 * S + 2 * NB + a); };
+    auto acc_empty_bar = [&](int a) { return bar_base + 8u * (2 * S + 2 * NB + 2 + a); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(sf_ready_bar(b), 4);
+            mbar_init(sf_free_bar(b), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(acc_full_bar(a), 1);
+            mbar_init(acc_empty_bar(a), 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 32) {
+        prefetch_tensor_map(&tmB);
+        prefetch_tensor_map(&tmA);
+        prefetch_tensor_map(&tmSB);
+        prefetch_tensor_map(&tmSA);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    grid_launch_dependents();
+    grid_dependency_wait();
+
+    JobCursor job;
+    job.init(prm);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();   // each weight tile is read by one unit
+            const uint64_t pol_a = policy_evict_last();    // token rows are shared by all N tiles
+            int it = 0;
+            for (; job.valid(); job.next()) {
+                const int nbox = (job.q_rows() + 15) / 16;
+                const int brow = job.g * prm.N + job.nt * kBM;   // row of B viewed as [G*N][K/2]
+                for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait(empty_bar(s), ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag)) goto producer_done;
+                    const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + 16 * kBM + nbox * (16 * kStageKBytes + 16 * 16));
+                    tma_load_2d(st, &tmB, full_bar(s), kt * kStageKBytes, brow, pol_w);
+                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSB, full_bar(s), kt * 16, brow, pol_w);
+                    for (int bx = 0; bx < nbox; ++bx) {
+                        tma_load_2d(st + C::P_BYTES + bx * 16 * kStageKBytes, &tmA, full_bar(s), kt * kStageKBytes,
+                                    job.q_row0() + 16 * bx, pol_a);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + bx * 256, &tmSA, full_bar(s),
+                                    kt * 16, job.q_row0() + 16 * bx, pol_a);
+                    }
+                }
+            }
+        producer_done:;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int it = 0, jc = 0;
+            for (; job.valid(); job.next(), ++jc) {
+                const int acc = jc & 1;
+                const uint32_t n_mma = (uint32_t)((job.q_rows() + 15) / 16 * 16);
+                const uint32_t idesc = idesc_nvf4(kBM, (int)n_mma);
+                if (!mbar_wait(acc_empty_bar(acc), ((uint32_t)(jc >> 1) & 1u) ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + acc * C::ACC_COLS;
+                bool ok = true;
+                for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
+                    const int s = it % S, b = it % NB;
+                    if (!mbar_wait(sf_ready_bar(b), (uint32_t)(it / NB) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                    const uint32_t sf = tmem + C::SF_BASE + b * C::SF_STRIDE;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        tc_mma_nvf4(d_tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
+                                    idesc, sf + 4 * j, sf + 16 + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                    tc_commit(empty_bar(s));
+                    tc_commit(sf_free_bar(b));
+                }
+                tc_commit(acc_full_bar(acc));
+                if (!ok) break;
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ---- scale writers (warp w owns TMEM lane quadrant w % 4)
+        const int quad = warp & 3;
+        const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+        int it = 0;
+        bool ok = true;
+        for (; ok && job.valid(); job.next()) {
+            for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
+                const int s = it % S, b = it % NB, use = it / NB;
+                int got = 1;
+                if (lane == 0)
+                    got = mbar_wait(full_bar(s), (uint32_t)(it / S) & 1u, abort_flag) &&
+                          (use == 0 || mbar_wait(sf_free_bar(b), (uint32_t)(use - 1) & 1u, abort_flag));
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                const uint32_t sf = t_quad + C::SF_BASE + b * C::SF_STRIDE;
+                uint32_t wp[16], wq[16];
+                gather_scale_words<true>(st + C::P_BYTES + C::Q_BYTES, lane, wp);
+                gather_scale_words<true>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq);
+                tmem_store_16(sf, wp);
+                tmem_store_16(sf + 16, wq);
+                tmem_wait_store();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sf_ready_bar(b));
+            }
+        }
+    } else {
+        // ---- epilogue (warps 2..5, TMEM lane quadrant w % 4 = weight rows)
+        const int quad = warp & 3;
+        const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+        int jc = 0;
+        for (; job.valid(); job.next(), ++jc) {
+            const int acc = jc & 1;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(acc_full_bar(acc), (uint32_t)(jc >> 1) & 1u, abort_flag) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, ok, 0) || *abort_flag) break;
+            tc_fence_after();
+            const int n = job.nt * kBM + quad * 32 + lane;     // output column
+            const int q0 = job.q_row0(), nq = job.q_rows();
+            const float alpha = __ldg(prm.alpha + job.g);
+#pragma unroll 1
+            for (int c0 = 0; c0 < nq; c0 += 16) {
+                uint32_t r[16];
+                tmem_load_16(t_quad + acc * C::ACC_COLS + c0, r);
+                tmem_wait_load();
+                if (n < prm.N) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (c0 + c < nq)
+                            prm.D[(size_t)(q0 + c0 + c) * prm.N + n] = __float2bfloat16_rn(__uint_as_float(r[c]) * alpha);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty_bar(acc));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace nvfp4

@@ -62,6 +62,9 @@ def test_gemm_argument_validation(L):
     assert L.nvfp4_gemm(None, p, p, p, 1.0, p, 4, 8, 128, None) == 1
     assert L.nvfp4_gemm(p, p, p, p, 1.0, None, 4, 8, 128, None) == 1
     assert L.nvfp4_gemm(odd, p, p, p, 1.0, p, 4, 8, 128, None) == 1
+    # gemm_ex flags
+    assert L.nvfp4_gemm_ex(p, p, p, p, 1.0, p, 4, 8, 96, 1, None) == 2
+    assert L.nvfp4_gemm_ex(p, p, p, p, 1.0, p, 4, 8, 128, 2, None) == 1
     # grouped
     assert L.nvfp4_grouped_gemm(p, p, p, p, p, p, 0, p, 4, 8, 128, None) == 1
     assert L.nvfp4_grouped_gemm(p, p, p, p, None, p, 2, p, 4, 8, 128, None) == 1

@@ -220,3 +220,39 @@ def test_gemm_unaligned_scales_take_the_relayout_path(nv):
     D = nv.gemm(dev(ca), sA, dev(cb), dev(sb), alpha)
     torch.cuda.synchronize()
     assert not violations(D.float().cpu().numpy(), ref, ad).any()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 768, 6144), (16, 256, 1024), (200, 264, 512), (512, 768, 2048)])
+def test_gemm_b_constant_prefetch_matches_oracle(nv, M, N, K):
+    # nvfp4_gemm_ex with the constant-B flag starts loading B before the
+    # previous kernel on the stream has finished; results must not change.
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "moe", 81 + M)
+    _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+    A, SA, B, SB = dev(ca), dev(sa), dev(cb), dev(sb)
+    outs = []
+    for _ in range(3):      # back-to-back launches exercise the early start
+        outs.append(nv.gemm(A, SA, B, SB, alpha, b_constant=True))
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    for D in outs:
+        assert not violations(D.float().cpu().numpy(), ref, ad).any()
+
+
+def test_gemm_b_constant_after_producer_of_A(nv):
+    # A is written by the kernel right before the GEMM; with the flag only B
+    # may be read early, so D must reflect the new A.
+    M, N, K = 8, 768, 2048
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "normal", 91)
+    ca2, sa2, _, _, _ = quantized_problem(M, N, K, "normal", 92)
+    _, ref2, ad2 = oracle.gemm(ca2, sa2, cb, sb, alpha, M, N, K)
+    A, SA, B, SB = dev(ca), dev(sa), dev(cb), dev(sb)
+    A2, SA2 = dev(ca2), dev(sa2)
+    for _ in range(3):
+        nv.gemm(A, SA, B, SB, alpha, b_constant=True)
+        A.copy_(A2)
+        SA.copy_(SA2)
+        D = nv.gemm(A, SA, B, SB, alpha, b_constant=True)
+        torch.cuda.synchronize()
+        assert not violations(D.float().cpu().numpy(), ref2, ad2).any()
+        A.copy_(dev(ca))
+        SA.copy_(dev(sa))
