@@ -30,6 +30,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from nvfp4_block_scaled_gemm_b200 import accounting, synth  # noqa: E402
+from nvfp4_block_scaled_gemm_b200.dist_timing import max_over_ranks  # noqa: E402
 
 METRIC = "NVFP4 GEMM TFLOPS & HBM GB/s vs B200 roofline, M-sweep on attn/MoE shapes"
 SWEEP_M = synth.ATTN_SWEEP_M
@@ -251,11 +252,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     clock_rec = clocks.stop(t_wall0, t_wall1)
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     status = nv.get_device_error(stream)
     if status != 0:
         raise RuntimeError(f"device error status {status}")
@@ -414,6 +411,120 @@ def run_reference(args):
     }
 
 
+# ---------------------------------------------------------------- other configurations
+def time_single_shape(nv, torch, dev, M, Nn, Kk, kind, seed, iters, stream, b_constant=False):
+    """Back-to-back GEMMs of one shape from a CUDA graph over rotating
+    buffers (> 4x L2); returns microseconds per GEMM."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    if kind == "uniform":
+        A32 = torch.rand((M, Kk), generator=gen, device=dev) * 2 - 1
+        B32 = torch.rand((Nn, Kk), generator=gen, device=dev) * 2 - 1
+    else:
+        A32 = torch.randn((M, Kk), generator=gen, device=dev)
+        B32 = torch.randn((Nn, Kk), generator=gen, device=dev) * (0.02 if kind == "moe" else 1.0)
+        if kind == "moe":
+            A32 = torch.where(torch.rand((M, Kk), generator=gen, device=dev) < 0.01, A32 * 20, A32)
+    a, sa, ga = nv.quantize(A32)
+    b, sb, gb = nv.quantize(B32)
+    del A32, B32
+    alpha = float(ga.item() * gb.item())
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nbytes = accounting.gemm_bytes(M, Nn, Kk)
+    R = int(max(2, min(64, -(-4 * l2 // nbytes))))
+    sets = [(a.clone(), sa.clone(), b.clone(), sb.clone(), torch.empty((M, Nn), dtype=torch.bfloat16, device=dev))
+            for _ in range(R)]
+    with torch.cuda.stream(stream):
+        for x in sets:
+            nv.gemm(x[0], x[1], x[2], x[3], alpha, out=x[4], stream=stream, b_constant=b_constant)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for x in sets:
+            nv.gemm(x[0], x[1], x[2], x[3], alpha, out=x[4], stream=stream, b_constant=b_constant)
+    reps = max(1, iters // R)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    assert nv.get_device_error(stream) == 0
+    return e0.elapsed_time(e1) * 1e3 / (reps * R)
+
+
+def run_shapes(args, shapes, label):
+    import torch
+    import nvfp4_block_scaled_gemm_b200 as nv
+    dev = torch.device("cuda", 0)
+    nv.lib()
+    hbm_gbs, bf16_tf, src = load_peaks()
+    fp4_tf = 4.0 * bf16_tf      # dense FP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
+    stream = torch.cuda.Stream()
+    rows = []
+    for (name, M, Nn, Kk, kind, seed) in shapes:
+        us = time_single_shape(nv, torch, dev, M, Nn, Kk, kind, seed, args.steps, stream)
+        b, f = accounting.gemm_bytes(M, Nn, Kk), accounting.gemm_flops(M, Nn, Kk)
+        t_roof = max(b / (hbm_gbs * 1e9), f / (fp4_tf * 1e12))
+        rows.append({"name": name, "M": M, "N": Nn, "K": Kk, "us": round(us, 2), "GBps": round(b / us / 1e3, 1),
+                     "TFLOPS": round(f / us / 1e6, 1), "roofline_frac": round(t_roof / (us * 1e-6), 4),
+                     "bound": "hbm" if b / (hbm_gbs * 1e9) >= f / (fp4_tf * 1e12) else "tensor"})
+    return {"workload": label, "peaks": {"hbm_gbs": hbm_gbs, "fp4_tflops": fp4_tf, "source": f"{src} (fp4 = 4 x bf16)"},
+            "shapes": rows}
+
+
+def run_grouped(args):
+    import torch
+    import nvfp4_block_scaled_gemm_b200 as nv
+    dev = torch.device("cuda", 0)
+    nv.lib()
+    hbm_gbs, bf16_tf, src = load_peaks()
+    G, Nn, Kk = synth.MOE_EXPERTS, synth.MOE_N, synth.HIDDEN_K
+    r = synth.moe_routing()
+    Mt = int(r.row_offsets[-1])
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1400)
+    X = torch.randn((synth.MOE_TOKENS, Kk), generator=gen, device=dev)
+    X = torch.where(torch.rand(X.shape, generator=gen, device=dev) < 0.01, X * 20, X)
+    ct, st_, ga = nv.quantize(X)
+    tok = torch.from_numpy(r.token_of_row.astype(np.int64)).to(dev)
+    A, sA = ct[tok].contiguous(), st_[tok].contiguous()
+    B = torch.empty((G, Nn, Kk // 2), dtype=torch.uint8, device=dev)
+    sB = torch.empty((G, Nn, Kk // 16), dtype=torch.uint8, device=dev)
+    alpha = torch.empty((G,), dtype=torch.float32, device=dev)
+    for g in range(G):
+        W = torch.randn((Nn, Kk), generator=gen, device=dev) * 0.02
+        cb, sb, gb = nv.quantize(W)
+        B[g].copy_(cb)
+        sB[g].copy_(sb)
+        alpha[g] = ga[0] * gb[0]
+    off = torch.from_numpy(r.row_offsets.astype(np.int32)).to(dev)
+    D = torch.empty((Mt, Nn), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        nv.grouped_gemm(A, sA, B, sB, alpha, off, out=D)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    iters = max(3, min(args.steps, 50))
+    e0.record()
+    for _ in range(iters):
+        nv.grouped_gemm(A, sA, B, sB, alpha, off, out=D)
+    e1.record()
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    us = e0.elapsed_time(e1) * 1e3 / iters
+    counts = [int(c) for c in np.diff(r.row_offsets)]
+    b, f = accounting.grouped_bytes(counts, Nn, Kk), accounting.grouped_flops(counts, Nn, Kk)
+    return {"workload": "grouped MoE: 256 experts x [2048 x 6144], 512 tokens top-8 Zipf(1.1) -> 4096 rows",
+            "active_experts": sum(1 for c in counts if c > 0), "max_rows": max(counts),
+            "us": round(us, 2), "GBps": round(b / us / 1e3, 1), "TFLOPS": round(f / us / 1e6, 2),
+            "hbm_frac": round(b / us / 1e3 / hbm_gbs, 4), "bytes": b, "peak_hbm_gbs": hbm_gbs,
+            "note": "weights stream once per launch (1.8 GB >> L2); eager launches, events"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -421,6 +532,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped"], default="attn",
+                    help="attn (default) prints the benchmark line; the others print a per-shape report")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -432,6 +545,14 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.workload != "attn":
+        if rank == 0:
+            if args.workload == "grouped":
+                print(json.dumps(run_grouped(args)), flush=True)
+            else:
+                shapes = synth.moe_sweep() if args.workload == "moe" else synth.saturation_sweep()
+                print(json.dumps(run_shapes(args, shapes, args.workload)), flush=True)
         return
 
     if world > 1:
