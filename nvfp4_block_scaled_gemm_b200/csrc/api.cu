@@ -180,7 +180,7 @@ PlanOverride plan_override() {
     const char* e = std::getenv("NVFP4_GEMM_PLAN");
     int a, b, c;
     if (e && std::sscanf(e, "%d:%d:%d", &a, &b, &c) == 3 && (b == 16 || b == 32 || b == 64 || b == 128 || b == 256) &&
-        (c == 1 || c == 2 || c == 4 || c == 8)) {
+        (c == 1 || c == 2 || c == 4 || c == 8 || c == 16)) {
         o.set = true;
         o.swap = a != 0;
         o.bq = b;
@@ -234,12 +234,15 @@ struct Maps {
 template <int BQ, bool SWAP, bool SPLITK, bool SFR>
 nvfp4_status launch_gemm_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, const GemmParams& prm, dim3 grid,
                                 cudaStream_t stream) {
-    using C = TileConfig<BQ>;
+    using C = TileConfig<BQ, SPLITK>;
     auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK, SFR>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!(info->smem_attr_set & bit)) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            // clusters of 16 split-K CTAs are opt-in (beyond the portable 8)
+            if (SPLITK && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
                 return NVFP4_ERR_CUDA;
             info->smem_attr_set |= bit;
         }

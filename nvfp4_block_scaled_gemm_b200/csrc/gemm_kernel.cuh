@@ -36,9 +36,12 @@
 // Split-K: the CTAs that share an output tile form one thread-block cluster
 // (blockIdx.x = cluster rank = K slice).  Rank r owns rows [r*128/S,
 // (r+1)*128/S) of the tile.  Every CTA stores each fp32 partial row straight
-// from registers into the owner's shared memory (distributed shared memory,
-// slot = the sender's rank); after one cluster barrier each owner sums its S
-// slots in rank order (deterministic), applies alpha and stores BF16.
+// from registers into the owner's receive slots (distributed shared memory,
+// slot = the sender's rank; a region of its own, outside the ring); after one
+// cluster barrier each owner sums its S slots in rank order (deterministic),
+// applies alpha and stores BF16.  The cluster barrier that guarantees every
+// peer has started is arrived at kernel start and waited on just before the
+// first remote store.
 //
 // Barriers: full[s] (producer arrive + TMA bytes), empty[s] (MMA commit:
 // stage s may be refilled), sf_ready[b] (4 writer arrivals: scale buffer b
@@ -61,7 +64,7 @@ constexpr int kThreads = 192;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 constexpr int kScaleBuffers = 4;    // rotating TMEM scale buffers
 
-template <int BQ>
+template <int BQ, bool SPLITK>
 struct TileConfig {
     static_assert(BQ == 16 || BQ == 32 || BQ == 64 || BQ == 128 || BQ == 256, "BQ");
     static constexpr int P_BYTES = kBM * kStageKBytes;
@@ -70,9 +73,16 @@ struct TileConfig {
     static constexpr int SFP_BYTES = 4 * kAtomBytes;
     static constexpr int SFQ_BYTES = 4 * kAtomBytes * Q_BLOCKS;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
-    static constexpr int STAGES_FIT = (kSmemLimit - 2048) / STAGE_BYTES;
+    // split-K receive slots: one fp32 row of kPartLd floats per tile row, in
+    // a region of their own when that still leaves at least 3 stages,
+    // otherwise in the ring (then written only after the whole cluster's
+    // main loops are done).
+    static constexpr int SLOT_NEED = kBM * (BQ + 4) * 4;
+    static constexpr bool OWN_SLOTS = SPLITK && (kSmemLimit - 2048 - SLOT_NEED) / STAGE_BYTES >= 3;
+    static constexpr int SLOT_BYTES = OWN_SLOTS ? SLOT_NEED : 0;
+    static constexpr int STAGES_FIT = (kSmemLimit - 2048 - SLOT_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SLOT_BYTES + 1024;
     // TMEM columns: fp32 accumulator [0, BQ), then kScaleBuffers scale buffers
     // of (P: 4 steps x 4) + (Q: 4 steps x 4 x Q_BLOCKS) columns.
     static constexpr int SF_BASE = BQ < 32 ? 32 : BQ;
@@ -149,6 +159,12 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t cluster_rank_addr(uint32_t smem_addr_local, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr_local), "r"(rank));
@@ -210,12 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                       const GemmParams prm) {
-    using C = TileConfig<BQ>;
+    using C = TileConfig<BQ, SPLITK>;
     constexpr int S = C::STAGES;
     constexpr int NB = kScaleBuffers;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+    // [ring: S stages][split-K receive slots][barriers]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES + C::SLOT_BYTES);
     // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB,2S+2NB) sf_free, [2S+2NB] accum
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -271,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (SPLITK) cluster_arrive_relaxed();   // "this CTA has started" (waited on before the push)
     // Everything above overlaps the previous kernel's tail when launched with
     // programmatic stream serialisation; global memory is touched only below.
     grid_launch_dependents();
@@ -281,8 +299,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // The 128-row side is read by exactly one tile column in the
             // swapped layout (the weights): stream it; keep the shared side.
-            const uint64_t pol_p = SWAP ? policy_evict_first() : policy_evict_last();
-            const uint64_t pol_q = SWAP ? policy_evict_last() : policy_evict_first();
+            // Swapped (small M): the weights P are read by exactly one tile
+            // column -- stream them; the few activation rows Q are shared by
+            // every CTA -- keep them.  Otherwise the row block P is shared by
+            // the CTAs of one wave and the column block Q by every wave.
+            const uint64_t pol_p = SWAP ? policy_evict_first() : policy_evict_normal();
+            const uint64_t pol_q = policy_evict_last();
             // With a constant B, its first ring's worth of tiles is requested
             // before waiting for the previous grid (only B is touched then).
             int pre = 0;
@@ -374,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;               // TMEM lane quadrant of this warp
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
         // ---- scale writers: shared memory -> TMEM scale buffer, per K tile.
-        // When the next K tile has landed too, both are written before the one
-        // tcgen05.wait::st, halving the store round trips.
+        // K tiles that have already landed (up to half the buffers) are
+        // written before one tcgen05.wait::st, sharing the store round trip.
         {
             int it = 0;
             for (int kt = kt_begin; kt < kt_end;) {
@@ -384,11 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int s0 = it % S, b0 = it % NB, use0 = it / NB;
                     got = mbar_wait(full_bar(s0), (uint32_t)(it / S) & 1u, abort_flag) &&
                           (use0 == 0 || mbar_wait(sf_free_bar(b0), (uint32_t)(use0 - 1) & 1u, abort_flag));
-                    if (got && kt + 1 < kt_end) {
-                        const int i1 = it + 1, s1 = i1 % S, b1 = i1 % NB, use1 = i1 / NB;
-                        if (mbar_test(full_bar(s1), (uint32_t)(i1 / S) & 1u) &&
-                            (use1 == 0 || mbar_test(sf_free_bar(b1), (uint32_t)(use1 - 1) & 1u)))
-                            cnt = 2;
+                    // take the following K tiles that have landed too, up to half
+                    // the scale buffers, so the MMA keeps the other half busy
+                    while (got && cnt < NB / 2 && kt + cnt < kt_end) {
+                        const int i1 = it + cnt, s1 = i1 % S, b1 = i1 % NB, use1 = i1 / NB;
+                        if (!mbar_test(full_bar(s1), (uint32_t)(i1 / S) & 1u) ||
+                            (use1 != 0 && !mbar_test(sf_free_bar(b1), (uint32_t)(use1 - 1) & 1u)))
+                            break;
+                        ++cnt;
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
@@ -451,16 +476,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (SPLITK) {
-        // Every CTA of the cluster is past its main loop (its accumulator is
-        // final, its ring idle): rows may now be pushed into peers' rings.
-        cluster_sync();
+        if (C::OWN_SLOTS) {
+            cluster_wait();   // every peer has started: its receive slots may be written
+        } else {
+            cluster_wait();
+            cluster_sync();   // every peer is past its main loop: its ring may be written
+        }
+        const uint32_t slots = C::OWN_SLOTS ? smem_base + S * C::STAGE_BYTES : smem_base;
         if (warp >= 2 && !*abort_flag) {
             const int quad = warp & 3;
             const int row = quad * 32 + lane;
             const int rows_per = kBM / splits;
             const uint32_t owner = (uint32_t)(row / rows_per);
-            const uint32_t local =
-                smem_base + (uint32_t)((split * rows_per + row % rows_per) * kPartLd<BQ>) * 4u;
+            const uint32_t local = slots + (uint32_t)((split * rows_per + row % rows_per) * kPartLd<BQ>) * 4u;
             const uint32_t dst = cluster_rank_addr(local, owner);
             const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
 #pragma unroll 1
@@ -473,8 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     st_cluster_v4(dst + 4u * (c0 + c), r[c], r[c + 1], r[c + 2], r[c + 3]);
             }
         }
-        cluster_sync();   // every partial row has reached its owner
-        if (warp >= 2 && !*abort_flag) reduce_owned_rows<BQ, SWAP>(prm, smem_base, tp, q_row0, threadIdx.x - 64);
+        cluster_sync();   // every partial row has reached its owner; no remote access after this
+        if (warp >= 2 && !*abort_flag) reduce_owned_rows<BQ, SWAP>(prm, slots, tp, q_row0, threadIdx.x - 64);
     }
 
     tc_fence_before();

@@ -256,3 +256,20 @@ def test_gemm_b_constant_after_producer_of_A(nv):
         assert not violations(D.float().cpu().numpy(), ref2, ad2).any()
         A.copy_(dev(ca))
         SA.copy_(dev(sa))
+
+
+@pytest.mark.parametrize("plan,M,N,K", [
+    ("1:16:16", 8, 768, 6144),     # 16-CTA split-K cluster (non-portable size)
+    ("0:256:8", 512, 512, 4096),   # 256-wide tiles, split-K slots in the ring
+    ("1:64:4", 100, 256, 2048),    # swapped, two token tiles
+    ("0:32:2", 300, 136, 1024),    # narrow tiles, ragged N
+    ("1:16:1", 40, 264, 512),      # swapped, three token tiles, no split
+])
+def test_gemm_forced_plans_match_oracle(nv, monkeypatch, plan, M, N, K):
+    # Every tile plan the dispatcher can take must give the same results.
+    monkeypatch.setenv("NVFP4_GEMM_PLAN", plan)
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "uniform", 101 + M)
+    _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+    got = run_gemm(nv, ca, sa, cb, sb, alpha)
+    bad = violations(got, ref, ad)
+    assert not bad.any(), f"{bad.sum()} outside the bound"
