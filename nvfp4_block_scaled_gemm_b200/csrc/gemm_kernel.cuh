@@ -44,9 +44,9 @@
 // first remote store.
 //
 // Barriers: full[s] (producer arrive + TMA bytes), empty[s] (MMA commit:
-// stage s may be refilled), sf_ready[b] (4 writer arrivals: scale buffer b
-// holds this K tile), sf_free[b] (MMA commit: buffer b may be rewritten),
-// accum (MMA commit after the last K tile).  Every wait is bounded.
+// stage s may be refilled and the TMEM scale buffer of that K tile may be
+// rewritten), sf_ready[b] (4 writer arrivals: scale buffer b holds this K
+// tile), accum (MMA commit after the last K tile).  Every wait is bounded.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -74,11 +74,11 @@ struct TileConfig {
     static constexpr int SFQ_BYTES = 4 * kAtomBytes * Q_BLOCKS;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
     // split-K receive slots: one fp32 row of kPartLd floats per tile row, in
-    // a region of their own when that still leaves at least 3 stages,
+    // a region of their own when that still leaves kScaleBuffers stages,
     // otherwise in the ring (then written only after the whole cluster's
     // main loops are done).
     static constexpr int SLOT_NEED = kBM * (BQ + 4) * 4;
-    static constexpr bool OWN_SLOTS = SPLITK && (kSmemLimit - 2048 - SLOT_NEED) / STAGE_BYTES >= 3;
+    static constexpr bool OWN_SLOTS = SPLITK && (kSmemLimit - 2048 - SLOT_NEED) / STAGE_BYTES >= kScaleBuffers;
     static constexpr int SLOT_BYTES = OWN_SLOTS ? SLOT_NEED : 0;
     static constexpr int STAGES_FIT = (kSmemLimit - 2048 - SLOT_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
@@ -92,7 +92,7 @@ struct TileConfig {
                                    : COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM columns");
     static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
-    static_assert(STAGES >= 2, "stages");
+    static_assert(STAGES >= kScaleBuffers, "scale buffers are released through the ring barriers");
 };
 
 struct GemmParams {
@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // [ring: S stages][split-K receive slots][barriers]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES + C::SLOT_BYTES);
-    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB,2S+2NB) sf_free, [2S+2NB] accum
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 1);
+    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB] accum
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + NB + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -249,8 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto full_bar = [&](int s) { return bar_base + 8u * s; };
     auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
     auto sf_ready_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
-    auto sf_free_bar = [&](int b) { return bar_base + 8u * (2 * S + NB + b); };
-    const uint32_t accum_bar = bar_base + 8u * (2 * S + 2 * NB);
+    const uint32_t accum_bar = bar_base + 8u * (2 * S + NB);
 
     // Q scale blocks that exist in the (row-padded) atom buffer for this tile.
     const int q_row0 = tq * BQ;
@@ -264,10 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int b = 0; b < NB; ++b) {
-            mbar_init(sf_ready_bar(b), 4);
-            mbar_init(sf_free_bar(b), 1);
-        }
+        for (int b = 0; b < NB; ++b) mbar_init(sf_ready_bar(b), 4);
         mbar_init(accum_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -384,8 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_nvf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
                                 idesc, sf + 4 * j, sf + 16 + 4 * C::Q_BLOCKS * j, (it > 0 || j > 0) ? 1u : 0u);
                 }
+                // one commit frees both the ring stage and the TMEM scale
+                // buffer this K tile used
                 tc_commit(empty_bar(s));
-                tc_commit(sf_free_bar(b));
             }
             // Always signal the epilogue (also after an abort), and only once
             // every MMA issued above has completed.
@@ -403,15 +400,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kt = kt_begin; kt < kt_end;) {
                 int got = 1, cnt = 1;
                 if (lane == 0) {
-                    const int s0 = it % S, b0 = it % NB, use0 = it / NB;
+                    // Scale buffer it % NB was last used by K tile it - NB; the MMA
+                    // commit on that tile's ring stage (empty) also releases it.
+                    // With NB <= S that barrier cannot run a phase ahead meanwhile.
+                    const int s0 = it % S, j0 = it - NB;
                     got = mbar_wait(full_bar(s0), (uint32_t)(it / S) & 1u, abort_flag) &&
-                          (use0 == 0 || mbar_wait(sf_free_bar(b0), (uint32_t)(use0 - 1) & 1u, abort_flag));
+                          (j0 < 0 || mbar_wait(empty_bar(j0 % S), (uint32_t)(j0 / S) & 1u, abort_flag));
                     // take the following K tiles that have landed too, up to half
                     // the scale buffers, so the MMA keeps the other half busy
                     while (got && cnt < NB / 2 && kt + cnt < kt_end) {
-                        const int i1 = it + cnt, s1 = i1 % S, b1 = i1 % NB, use1 = i1 / NB;
+                        const int i1 = it + cnt, s1 = i1 % S, j1 = i1 - NB;
                         if (!mbar_test(full_bar(s1), (uint32_t)(i1 / S) & 1u) ||
-                            (use1 != 0 && !mbar_test(sf_free_bar(b1), (uint32_t)(use1 - 1) & 1u)))
+                            (j1 >= 0 && !mbar_test(empty_bar(j1 % S), (uint32_t)(j1 / S) & 1u)))
                             break;
                         ++cnt;
                     }
