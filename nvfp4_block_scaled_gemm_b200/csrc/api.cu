@@ -17,6 +17,7 @@
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
 #include "grouped_kernel.cuh"
+#include "persistent_kernel.cuh"
 
 namespace {
 
@@ -291,6 +292,39 @@ nvfp4_status launch_by_bq(int bq, DeviceInfo* info, const Maps& m, const GemmPar
     }
 }
 
+// Persistent large-tile kernel: one CTA per SM walking the tile list.
+template <int BQ>
+nvfp4_status launch_persistent(DeviceInfo* info, uint64_t bit, const Maps& m, const nvfp4::PersistParams& prm,
+                               int tiles, cudaStream_t stream) {
+    using C = nvfp4::PersistConfig<BQ>;
+    auto kern = nvfp4::nvfp4_gemm_persistent_kernel<BQ>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(info->smem_attr_set & bit)) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            info->smem_attr_set |= bit;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(tiles, info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kPersistThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m.p, m.q, m.sp, m.sq, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
 template <bool SFR>
 nvfp4_status launch_mode(const Plan& plan, DeviceInfo* info, const Maps& m, const GemmParams& prm, dim3 grid,
                          cudaStream_t stream) {
@@ -445,6 +479,22 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     prm.k_tiles = plan.k_tiles;
     prm.tiles_q = plan.tiles_q;
     prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+    // More tiles than SMs, no split, row-major scales: the persistent kernel.
+    const int tiles = plan.tiles_p * plan.tiles_q;
+    if (sfr && !plan.swap && plan.splits == 1 && tiles > info->num_sms && (plan.bq == 128 || plan.bq == 256) &&
+        !plan_override().set) {
+        nvfp4::PersistParams pp{};
+        pp.D = static_cast<__nv_bfloat16*>(D);
+        pp.alpha = alpha;
+        pp.M = M;
+        pp.N = N;
+        pp.K = K;
+        pp.k_tiles = K / 256;
+        pp.tiles_m = plan.tiles_p;
+        pp.tiles_n = plan.tiles_q;
+        return plan.bq == 256 ? launch_persistent<256>(info, 1ull << 60, maps, pp, tiles, stream)
+                              : launch_persistent<128>(info, 1ull << 61, maps, pp, tiles, stream);
+    }
     const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
     return sfr ? launch_mode<true>(plan, info, maps, prm, grid, stream)
                : launch_mode<false>(plan, info, maps, prm, grid, stream);

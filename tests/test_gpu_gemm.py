@@ -273,3 +273,22 @@ def test_gemm_forced_plans_match_oracle(nv, monkeypatch, plan, M, N, K):
     got = run_gemm(nv, ca, sa, cb, sb, alpha)
     bad = violations(got, ref, ad)
     assert not bad.any(), f"{bad.sum()} outside the bound"
+
+
+@pytest.mark.parametrize("M,N,K,full", [
+    (1024, 2432, 256, True),      # 8 x 19 = 152 tiles of 128x128: persistent, BQ 128
+    (1100, 4104, 512, False),     # 9 x 17 = 153 tiles of 128x256, ragged M and N: persistent, BQ 256
+    (4096, 4096, 1024, False),    # 32 x 16 = 512 tiles, several tiles per CTA
+])
+def test_gemm_persistent_path_matches_oracle(nv, M, N, K, full):
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "uniform", 131 + M)
+    got = run_gemm(nv, ca, sa, cb, sb, alpha)
+    if full:
+        _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+        assert not violations(got, ref, ad).any()
+    else:
+        rng = np.random.default_rng(M + N)
+        rows = np.concatenate([rng.integers(0, M, 4000), [M - 1, M - 1, 0]])
+        cols = np.concatenate([rng.integers(0, N, 4000), [N - 1, 0, N - 1]])
+        _, ref, ad = oracle.gemm_sampled(ca, sa, cb, sb, alpha, M, N, K, rows, cols)
+        assert not violations(got[rows, cols], ref, ad).any()
