@@ -42,9 +42,11 @@ struct GroupedConfig {
     static constexpr int SFP_BYTES = 4 * kAtomBytes;
     static constexpr int SFQ_BYTES = 4 * kAtomBytes;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
-    static constexpr int STAGES = (kSmemLimit - 2048) / STAGE_BYTES;
+    static constexpr int STAGES_FIT = (kSmemLimit - 2048) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    static_assert(STAGES >= kScaleBuffers, "scale buffers are released through the ring barriers");
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
-    // TMEM: two accumulators [0,128) and [128,256), then 4 scale buffers of 32.
+    // TMEM: two accumulators [0,BQ) and [BQ,2BQ), then 4 scale buffers of 32.
     static constexpr int ACC_COLS = BQ;
     static constexpr int SF_BASE = 2 * BQ;
     static constexpr int SF_STRIDE = 32;
@@ -98,9 +100,9 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB,2S+2NB) sf_free,
-    //       [2S+2NB, +2) acc_full, [2S+2NB+2, +2) acc_empty
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 4);
+    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB, +2) acc_full,
+    //       [2S+NB+2, +2) acc_empty
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + NB + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,19 +111,15 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     auto full_bar = [&](int s) { return bar_base + 8u * s; };
     auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
     auto sf_ready_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
-    auto sf_free_bar = [&](int b) { return bar_base + 8u * (2 * S + NB + b); };
-    auto acc_full_bar = [&](int a) { return bar_base + 8u * (2 * S + 2 * NB + a); };
-    auto acc_empty_bar = [&](int a) { return bar_base + 8u * (2 * S + 2 * NB + 2 + a); };
+    auto acc_full_bar = [&](int a) { return bar_base + 8u * (2 * S + NB + a); };
+    auto acc_empty_bar = [&](int a) { return bar_base + 8u * (2 * S + NB + 2 + a); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int b = 0; b < NB; ++b) {
-            mbar_init(sf_ready_bar(b), 4);
-            mbar_init(sf_free_bar(b), 1);
-        }
+        for (int b = 0; b < NB; ++b) mbar_init(sf_ready_bar(b), 4);
         for (int a = 0; a < 2; ++a) {
             mbar_init(acc_full_bar(a), 1);
             mbar_init(acc_empty_bar(a), 4);
@@ -198,8 +196,7 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
                     for (int j = 0; j < 4; ++j)
                         tc_mma_nvf4(d_tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
                                     idesc, sf + 4 * j, sf + 16 + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
-                    tc_commit(empty_bar(s));
-                    tc_commit(sf_free_bar(b));
+                    tc_commit(empty_bar(s));   // frees the ring stage and scale buffer b
                 }
                 tc_commit(acc_full_bar(acc));
                 if (!ok) break;
@@ -214,11 +211,13 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         bool ok = true;
         for (; ok && job.valid(); job.next()) {
             for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
-                const int s = it % S, b = it % NB, use = it / NB;
+                const int s = it % S, b = it % NB, j = it - NB;
                 int got = 1;
+                // scale buffer b was last used by K tile it - NB, released by
+                // the MMA commit on that tile's ring stage
                 if (lane == 0)
                     got = mbar_wait(full_bar(s), (uint32_t)(it / S) & 1u, abort_flag) &&
-                          (use == 0 || mbar_wait(sf_free_bar(b), (uint32_t)(use - 1) & 1u, abort_flag));
+                          (j < 0 || mbar_wait(empty_bar(j % S), (uint32_t)(j / S) & 1u, abort_flag));
                 if (!__shfl_sync(0xffffffffu, got, 0)) {
                     ok = false;
                     break;
