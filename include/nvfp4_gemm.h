@@ -179,6 +179,34 @@ const char* nvfp4_status_string(nvfp4_status status);
  */
 nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/*
+ * nvfp4_gemm_noalloc -- the same GEMM as nvfp4_gemm (same arguments, layouts,
+ * requirements and result), for callers that are not allowed to allocate
+ * device memory during the call: runtimes that own and pool all device
+ * memory themselves, code that runs under a fixed memory budget, or callers
+ * that must keep driver allocations off their launch path.  nvfp4_gemm may
+ * cudaMalloc scratch on its first call of a new shape; this entry point never
+ * calls cudaMalloc, cudaFree or any allocating routine.  It has no counterpart
+ * on the source pages; it is a deployment convenience of this library.
+ *   Its one piece of scratch -- the operands' scales re-laid out for the
+ *   tensor cores -- is a static device array of 8 MiB (8,388,608 bytes) that
+ *   every GPU which loads the library keeps until the process exits.  Problems whose scales
+ *   need more, i.e. (ceil(M/128) + ceil(N/128)) * (K/64) * 512 bytes (plus up
+ *   to 255 bytes of alignment) above that limit, are rejected with
+ *   NVFP4_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before capturing the stream into a CUDA graph.
+ *   All calls share the one array, so calls whose work overlaps on the GPU
+ *   (different streams, or different host threads) race on it: serialise
+ *   them.  Each call rewrites every scratch byte it reads, so no clearing is
+ *   needed between calls.
+ */
+nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA,
+                                const void* B, const void* sB,
+                                float alpha, void* D,
+                                int M, int N, int K, void* stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int nvfp4_version(void);
 

@@ -32,6 +32,7 @@ EXPORTS = (
     "nvfp4_gemm", "nvfp4_gemm_ex", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
+    "nvfp4_gemm_noalloc",
 )
 
 
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).restype = i32
         L.nvfp4_version.restype = i32
         L.nvfp4_kernel_launches.restype = ctypes.c_ulonglong
+        L.nvfp4_gemm_noalloc.argtypes = [P, P, P, P, f32, P, i32, i32, i32, P]
+        L.nvfp4_gemm_noalloc.restype = i32
         _lib = L
     return _lib
 
@@ -132,6 +135,30 @@ def gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, a
     else:
         _check(lib().nvfp4_gemm(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
                                 out.data_ptr(), M, N, K, _stream(stream)), "nvfp4_gemm")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20   # static device scratch of nvfp4_gemm_noalloc
+
+
+def gemm_noalloc(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, alpha: float,
+                 out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Same as gemm(), through nvfp4_gemm_noalloc: the library allocates no
+    device memory (its scale scratch is a fixed static device array), so the
+    output tensor must be supplied.  Calls whose GPU work overlaps race on
+    that shared scratch; keep them serialised."""
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D packed E2M1 tensors [rows, K/2]")
+    M, N, K = A.shape[0], B.shape[0], packed_k(A)
+    if packed_k(B) != K:
+        raise ValueError(f"K mismatch: A holds K={K}, B holds K={packed_k(B)}")
+    _need(A, "A", torch.uint8, (M, K // 2))
+    _need(B, "B", torch.uint8, (N, K // 2))
+    _need(sA, "sA", torch.uint8, (M, K // 16))
+    _need(sB, "sB", torch.uint8, (N, K // 16))
+    _need(out, "out", torch.bfloat16, (M, N))
+    _check(lib().nvfp4_gemm_noalloc(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
+                                    out.data_ptr(), M, N, K, _stream(stream)), "nvfp4_gemm_noalloc")
     return out
 
 

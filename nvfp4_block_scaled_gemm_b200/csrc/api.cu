@@ -588,3 +588,97 @@ nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream_) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// GEMM without any device allocation (nvfp4_gemm_noalloc).
+//
+// For callers that may not allocate device memory at call time: hosts that
+// own every byte of device memory themselves (a serving runtime with its own
+// pool, a plugin inside another framework), code with a fixed memory budget,
+// or callers that must not trigger a driver allocation on the launch path.
+// nvfp4_gemm may cudaMalloc per-stream scratch on its first call of a shape;
+// this variant never does.  Its only scratch -- the scales re-laid out for
+// the tensor cores -- lives in the file-scope device array below, which every
+// GPU that loads this library holds for the life of the process.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB per device
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+std::map<int, uint8_t*> g_noalloc_addr;   // device -> device address of g_noalloc_scratch
+
+// The array's name in host code is only a host-side handle; the device
+// address has to be looked up, once per device, with that device current.
+nvfp4_status noalloc_scratch_address(int dev, uint8_t** out) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    auto it = g_noalloc_addr.find(dev);
+    if (it == g_noalloc_addr.end()) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        it = g_noalloc_addr.emplace(dev, static_cast<uint8_t*>(p)).first;
+    }
+    *out = it->second;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA, const void* B, const void* sB, float alpha, void* D,
+                                int M, int N, int K, void* stream_) {
+    nvfp4_status st = check_gemm_args(A, sA, B, sB, D, M, N, K);
+    if (st != NVFP4_OK || M == 0 || N == 0) return st;
+    // Scales of both operands, re-laid out, must fit the static scratch.
+    const size_t sfa_bytes = nvfp4_swizzled_scale_bytes(M, K);
+    const size_t sfb_bytes = nvfp4_swizzled_scale_bytes(N, K);
+    if (align_up(sfa_bytes, 256) + sfb_bytes > kNoAllocScratchBytes) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    int dev;
+    DeviceInfo* info;
+    st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    uint8_t* scratch = nullptr;
+    if ((st = noalloc_scratch_address(dev, &scratch)) != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+    const Plan plan = make_plan(M, N, K, info->num_sms, /*sfr=*/false);
+    const void* P = plan.swap ? B : A;
+    const void* Q = plan.swap ? A : B;
+    const void* sP = plan.swap ? sB : sA;
+    const void* sQ = plan.swap ? sA : sB;
+    const int rows_p = plan.swap ? N : M;
+    const int rows_q = plan.swap ? M : N;
+    uint8_t* sfp = scratch;
+    uint8_t* sfq = scratch + align_up(nvfp4_swizzled_scale_bytes(rows_p, K), 256);
+    // Every byte the kernel reads is rewritten by these two passes (padding
+    // rows included), so nothing left by an earlier call needs clearing.
+    if ((st = launch_swizzle(sP, rows_p, K, sfp, stream)) != NVFP4_OK) return st;
+    if ((st = launch_swizzle(sQ, rows_q, K, sfq, stream)) != NVFP4_OK) return st;
+
+    Maps maps;
+    if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq))
+        return NVFP4_ERR_CUDA;
+    maps.sp = maps.p;
+    maps.sq = maps.q;
+    GemmParams prm{};
+    prm.sfp = sfp;
+    prm.sfq = sfq;
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.alpha = alpha;
+    prm.rows_p = rows_p;
+    prm.rows_q = rows_q;
+    prm.K = K;
+    prm.ldd = N;
+    prm.k_tiles = plan.k_tiles;
+    prm.tiles_q = plan.tiles_q;
+    prm.prefetch_b = 0;
+    const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
+    return launch_mode<false>(plan, info, maps, prm, grid, stream);
+}
+
+}  // extern "C"
