@@ -17,6 +17,7 @@
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
 #include "grouped_kernel.cuh"
+#include "pair_kernel.cuh"
 #include "persistent_kernel.cuh"
 
 namespace {
@@ -35,6 +36,7 @@ struct DeviceInfo {
     bool supported = false;
     int num_sms = 0;
     uint64_t smem_attr_set = 0;  // bit per kernel instantiation
+    int pair_clusters = -1;      // co-resident 2-CTA clusters of the pair kernel (-1: not queried)
 };
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_devices;
@@ -325,6 +327,68 @@ nvfp4_status launch_persistent(DeviceInfo* info, uint64_t bit, const Maps& m, co
     return NVFP4_OK;
 }
 
+// Whether large problems use the CTA-pair kernel: NVFP4_GEMM_PAIR=0 turns it
+// off (the single-CTA persistent kernel runs instead), anything else or unset
+// leaves it on.
+bool pair_kernel_enabled() {
+    const char* e = std::getenv("NVFP4_GEMM_PAIR");
+    return !(e && e[0] == '0');
+}
+
+nvfp4_status launch_pair(DeviceInfo* info, const Maps& m, const nvfp4::PersistParams& prm, cudaStream_t stream) {
+    using C = nvfp4::PairConfig;
+    auto kern = nvfp4::nvfp4_gemm_pair_kernel;
+    int clusters;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(info->smem_attr_set & (1ull << 59))) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            info->smem_attr_set |= (1ull << 59);
+        }
+        if (info->pair_clusters < 0) {
+            // A persistent grid larger than what fits at once would serialise
+            // whole clusters: size it by the co-resident cluster count.
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(2, 1, 1);
+            q.blockDim = dim3(nvfp4::kPersistThreads, 1, 1);
+            q.dynamicSmemBytes = C::SMEM_BYTES;
+            cudaLaunchAttribute ca[1];
+            ca[0].id = cudaLaunchAttributeClusterDimension;
+            ca[0].val.clusterDim.x = 2;
+            ca[0].val.clusterDim.y = 1;
+            ca[0].val.clusterDim.z = 1;
+            q.attrs = ca;
+            q.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                return NVFP4_ERR_CUDA;
+            }
+            info->pair_clusters = n;
+        }
+        clusters = info->pair_clusters;
+    }
+    const int tiles = prm.tiles_m * prm.tiles_n;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * (unsigned)std::min(tiles, clusters), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kPersistThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m.p, m.q, m.sp, m.sq, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
 template <bool SFR>
 nvfp4_status launch_mode(const Plan& plan, DeviceInfo* info, const Maps& m, const GemmParams& prm, dim3 grid,
                          cudaStream_t stream) {
@@ -492,6 +556,17 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
         pp.k_tiles = K / 256;
         pp.tiles_m = plan.tiles_p;
         pp.tiles_n = plan.tiles_q;
+        if (plan.bq == 256 && M >= 256 && pair_kernel_enabled()) {
+            // 256 x 256 tiles on CTA pairs; the maps cover this CTA's 128 rows
+            // of A and of B and the scales of all 256 B rows.
+            Maps pm;
+            if (!make_operand_map(&pm.p, A, M, K / 2, 128) || !make_operand_map(&pm.q, B, N, K / 2, 128) ||
+                !make_scale_map(&pm.sp, sA, M, K / 16, 128) || !make_scale_map(&pm.sq, sB, N, K / 16, 256))
+                return NVFP4_ERR_CUDA;
+            pp.tiles_m = (M + nvfp4::kPairBM - 1) / nvfp4::kPairBM;
+            pp.tiles_n = (N + nvfp4::kPairBN - 1) / nvfp4::kPairBN;
+            return launch_pair(info, pm, pp, stream);
+        }
         return plan.bq == 256 ? launch_persistent<256>(info, 1ull << 60, maps, pp, tiles, stream)
                               : launch_persistent<128>(info, 1ull << 61, maps, pp, tiles, stream);
     }

@@ -275,20 +275,43 @@ def test_gemm_forced_plans_match_oracle(nv, monkeypatch, plan, M, N, K):
     assert not bad.any(), f"{bad.sum()} outside the bound"
 
 
+def boundary_samples(M, N, seed, n_random=4000, edge=256):
+    """Random (row, col) pairs plus every element of the rows and columns
+    that sit on either side of a 128/256 tile edge and at the ragged end."""
+    rng = np.random.default_rng(seed)
+    rows = [rng.integers(0, M, n_random)]
+    cols = [rng.integers(0, N, n_random)]
+    for r in sorted({0, 127, 128, min(255, M - 1), min(256, M - 1), M - 1}):
+        c = np.arange(0, N, max(1, N // edge))
+        rows.append(np.full(c.size, r))
+        cols.append(c)
+    for c in sorted({0, 127, 128, min(255, N - 1), min(256, N - 1), N - 1}):
+        r = np.arange(0, M, max(1, M // edge))
+        rows.append(r)
+        cols.append(np.full(r.size, c))
+    rows.append(np.array([M - 1, M - 1, 0]))
+    cols.append(np.array([N - 1, 0, N - 1]))
+    return np.concatenate(rows), np.concatenate(cols)
+
+
+@pytest.mark.parametrize("pair", ["1", "0"])
 @pytest.mark.parametrize("M,N,K,full", [
     (1024, 2432, 256, True),      # 8 x 19 = 152 tiles of 128x128: persistent, BQ 128
-    (1100, 4104, 512, False),     # 9 x 17 = 153 tiles of 128x256, ragged M and N: persistent, BQ 256
-    (4096, 4096, 1024, False),    # 32 x 16 = 512 tiles, several tiles per CTA
+    (1100, 4104, 512, False),     # 153 tiles of 128x256, ragged M and N: CTA-pair tiles of 256x256
+                                  # whose second half lies wholly past M (rows) and N (columns)
+    (4096, 4096, 1024, False),    # 32 x 16 = 512 tiles, several tiles per CTA (pair)
+    (2304, 4352, 2048, False),    # 9 x 17 pair tiles, long K
 ])
-def test_gemm_persistent_path_matches_oracle(nv, M, N, K, full):
+def test_gemm_persistent_path_matches_oracle(nv, monkeypatch, pair, M, N, K, full):
+    # NVFP4_GEMM_PAIR=0 selects the single-CTA persistent kernel where the
+    # CTA-pair kernel would run; both must give the oracle's results.
+    monkeypatch.setenv("NVFP4_GEMM_PAIR", pair)
     ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "uniform", 131 + M)
     got = run_gemm(nv, ca, sa, cb, sb, alpha)
     if full:
         _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
         assert not violations(got, ref, ad).any()
     else:
-        rng = np.random.default_rng(M + N)
-        rows = np.concatenate([rng.integers(0, M, 4000), [M - 1, M - 1, 0]])
-        cols = np.concatenate([rng.integers(0, N, 4000), [N - 1, 0, N - 1]])
+        rows, cols = boundary_samples(M, N, M + N)
         _, ref, ad = oracle.gemm_sampled(ca, sa, cb, sb, alpha, M, N, K, rows, cols)
         assert not violations(got[rows, cols], ref, ad).any()
