@@ -335,7 +335,8 @@ bool pair_kernel_enabled() {
     return !(e && e[0] == '0');
 }
 
-nvfp4_status launch_pair(DeviceInfo* info, const Maps& m, const nvfp4::PersistParams& prm, cudaStream_t stream) {
+nvfp4_status launch_pair(DeviceInfo* info, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                         const nvfp4::PairParams& prm, cudaStream_t stream) {
     using C = nvfp4::PairConfig;
     auto kern = nvfp4::nvfp4_gemm_pair_kernel;
     int clusters;
@@ -351,7 +352,7 @@ nvfp4_status launch_pair(DeviceInfo* info, const Maps& m, const nvfp4::PersistPa
             // whole clusters: size it by the co-resident cluster count.
             cudaLaunchConfig_t q = {};
             q.gridDim = dim3(2, 1, 1);
-            q.blockDim = dim3(nvfp4::kPersistThreads, 1, 1);
+            q.blockDim = dim3(nvfp4::kPairThreads, 1, 1);
             q.dynamicSmemBytes = C::SMEM_BYTES;
             cudaLaunchAttribute ca[1];
             ca[0].id = cudaLaunchAttributeClusterDimension;
@@ -372,7 +373,7 @@ nvfp4_status launch_pair(DeviceInfo* info, const Maps& m, const nvfp4::PersistPa
     const int tiles = prm.tiles_m * prm.tiles_n;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2u * (unsigned)std::min(tiles, clusters), 1, 1);
-    cfg.blockDim = dim3(nvfp4::kPersistThreads, 1, 1);
+    cfg.blockDim = dim3(nvfp4::kPairThreads, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -380,13 +381,50 @@ nvfp4_status launch_pair(DeviceInfo* info, const Maps& m, const nvfp4::PersistPa
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m.p, m.q, m.sp, m.sq, prm);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, prm);
     g_launches++;
     if (e != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
     }
     return NVFP4_OK;
+}
+
+// The CTA-pair kernel: scales re-laid out into tensor-core atoms in scratch,
+// then 256 x 256 tiles on CTA pairs.
+nvfp4_status pair_gemm(int dev, DeviceInfo* info, const void* A, const void* sA, const void* B, const void* sB,
+                       float alpha, void* D, int M, int N, int K, cudaStream_t stream) {
+    const size_t sfa_bytes = nvfp4_swizzled_scale_bytes(M, K);
+    const size_t off_sfb = align_up(sfa_bytes, 256);
+    const size_t sfb_bytes = nvfp4_swizzled_scale_bytes(N, K);
+    uint8_t* ws = nullptr;
+    nvfp4_status st = get_scratch(dev, stream, off_sfb + sfb_bytes, &ws);
+    if (st != NVFP4_OK) return st;
+    CUtensorMap tmA, tmB;
+    if (!make_operand_map(&tmA, A, M, K / 2, 128) || !make_operand_map(&tmB, B, N, K / 2, 128)) return NVFP4_ERR_CUDA;
+    {
+        nvfp4::ScaleTileJob ja{static_cast<const uint8_t*>(sA), ws, M, (M + 127) / 128, aligned(sA, 16) ? 1 : 0};
+        nvfp4::ScaleTileJob jb{static_cast<const uint8_t*>(sB), ws + off_sfb, N, (N + 127) / 128,
+                               aligned(sB, 16) ? 1 : 0};
+        const long long blocks = (long long)(ja.row_blocks + jb.row_blocks) * (K / 256);
+        nvfp4::swizzle_scale_tiles_kernel<<<(unsigned)blocks, 128, 0, stream>>>(ja, jb, K / 16, K / 256);
+        g_launches++;
+        if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    nvfp4::PairParams pp{};
+    pp.D = static_cast<__nv_bfloat16*>(D);
+    pp.sfa = ws;
+    pp.sfb = ws + off_sfb;
+    pp.alpha = alpha;
+    pp.M = M;
+    pp.N = N;
+    pp.K = K;
+    pp.k_tiles = K / 256;
+    pp.tiles_m = (M + nvfp4::kPairBM - 1) / nvfp4::kPairBM;
+    pp.tiles_n = (N + nvfp4::kPairBN - 1) / nvfp4::kPairBN;
+    pp.rb_a = (M + 127) / 128;
+    pp.rb_b = (N + 127) / 128;
+    return launch_pair(info, tmA, tmB, pp, stream);
 }
 
 template <bool SFR>
@@ -501,6 +539,10 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     // scratch first.
     const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
     const Plan plan = make_plan(M, N, K, info->num_sms, sfr);
+    // Many 256-wide tiles: the CTA-pair kernel.
+    if (K % 256 == 0 && !plan.swap && plan.splits == 1 && plan.bq == 256 && M >= 256 &&
+        plan.tiles_p * plan.tiles_q > info->num_sms && pair_kernel_enabled() && !plan_override().set)
+        return pair_gemm(dev, info, A, sA, B, sB, alpha, D, M, N, K, stream);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
     const void* sP = plan.swap ? sB : sA;
@@ -556,17 +598,6 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
         pp.k_tiles = K / 256;
         pp.tiles_m = plan.tiles_p;
         pp.tiles_n = plan.tiles_q;
-        if (plan.bq == 256 && M >= 256 && pair_kernel_enabled()) {
-            // 256 x 256 tiles on CTA pairs; the maps cover this CTA's 128 rows
-            // of A and of B and the scales of all 256 B rows.
-            Maps pm;
-            if (!make_operand_map(&pm.p, A, M, K / 2, 128) || !make_operand_map(&pm.q, B, N, K / 2, 128) ||
-                !make_scale_map(&pm.sp, sA, M, K / 16, 128) || !make_scale_map(&pm.sq, sB, N, K / 16, 256))
-                return NVFP4_ERR_CUDA;
-            pp.tiles_m = (M + nvfp4::kPairBM - 1) / nvfp4::kPairBM;
-            pp.tiles_n = (N + nvfp4::kPairBN - 1) / nvfp4::kPairBN;
-            return launch_pair(info, pm, pp, stream);
-        }
         return plan.bq == 256 ? launch_persistent<256>(info, 1ull << 60, maps, pp, tiles, stream)
                               : launch_persistent<128>(info, 1ull << 61, maps, pp, tiles, stream);
     }

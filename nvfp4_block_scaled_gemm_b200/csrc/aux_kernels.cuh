@@ -30,6 +30,49 @@ __global__ void swizzle_scales_kernel(const uint8_t* __restrict__ s, int rows, i
     *reinterpret_cast<uint4*>(out + (rb * steps + ks) * 512 + 16 * L) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// The same layout for two scale tensors in one launch, K a multiple of 256:
+// one 128-thread CTA per (tensor, 128-row block, 256-element K tile).  Thread
+// t reads the 16 scale bytes of row t of the block (one request per row), the
+// CTA transposes them through shared memory and writes the four 512-byte
+// atoms of the K tile as contiguous, fully coalesced lines.
+struct ScaleTileJob {
+    const uint8_t* s;   // row-major [rows][K/16]
+    uint8_t* out;       // atoms [ceil(rows/128)][K/64][512 B]
+    int rows;
+    int row_blocks;     // ceil(rows / 128)
+    int vec16;          // s and its rows are 16-byte aligned
+};
+
+__global__ void __launch_bounds__(128) swizzle_scale_tiles_kernel(ScaleTileJob a, ScaleTileJob b, int kb_row,
+                                                                  int k_tiles) {
+    __shared__ uint32_t tile[128][5];   // odd row pitch: conflict-free column reads
+    int blk = (int)blockIdx.x;
+    const int blocks_a = a.row_blocks * k_tiles;
+    const ScaleTileJob& job = blk < blocks_a ? a : b;
+    if (blk >= blocks_a) blk -= blocks_a;
+    const int rb = blk / k_tiles, kt = blk - rb * k_tiles;
+    const int t = (int)threadIdx.x;
+    const long long r = (long long)rb * 128 + t;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (r < job.rows) {
+        const uint8_t* src = job.s + r * kb_row + 16 * kt;
+        if (job.vec16) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
+            w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = __ldg(reinterpret_cast<const uint32_t*>(src) + j);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tile[t][j] = w[j];
+    __syncthreads();
+    const int j = t >> 5, L = t & 31;   // warp j writes the atom of K step 4*kt + j
+    const size_t steps = (size_t)k_tiles * 4;
+    uint8_t* atom = job.out + ((size_t)rb * steps + 4 * (size_t)kt + j) * 512;
+    *reinterpret_cast<uint4*>(atom + 16 * L) = make_uint4(tile[L][j], tile[L + 32][j], tile[L + 64][j], tile[L + 96][j]);
+}
+
 // ------------------------------------------------------------ quantization
 // Pass 1: amax over the tensor, as the bit pattern of a non-negative float
 // (monotone as an unsigned integer) accumulated with atomicMax.

@@ -222,6 +222,26 @@ def test_gemm_unaligned_scales_take_the_relayout_path(nv):
     assert not violations(D.float().cpu().numpy(), ref, ad).any()
 
 
+def test_gemm_pair_path_unaligned_scales(nv):
+    # The CTA-pair kernel re-lays both scale tensors out into atoms on the
+    # device; with sA and sB only 4-byte aligned the re-layout reads them a
+    # word at a time.
+    M, N, K = 2304, 4352, 512
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "moe", 73)
+    bufa = torch.zeros(sa.size + 4, dtype=torch.uint8, device="cuda")
+    bufb = torch.zeros(sb.size + 4, dtype=torch.uint8, device="cuda")
+    sA = bufa[4:].view(M, K // 16)
+    sB = bufb[4:].view(N, K // 16)
+    sA.copy_(dev(sa))
+    sB.copy_(dev(sb))
+    D = nv.gemm(dev(ca), sA, dev(cb), sB, alpha)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    rows, cols = boundary_samples(M, N, 77)
+    _, ref, ad = oracle.gemm_sampled(ca, sa, cb, sb, alpha, M, N, K, rows, cols)
+    assert not violations(D.float().cpu().numpy()[rows, cols], ref, ad).any()
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 768, 6144), (16, 256, 1024), (200, 264, 512), (512, 768, 2048)])
 def test_gemm_b_constant_prefetch_matches_oracle(nv, M, N, K):
     # nvfp4_gemm_ex with the constant-B flag starts loading B before the
