@@ -539,9 +539,10 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     // scratch first.
     const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
     const Plan plan = make_plan(M, N, K, info->num_sms, sfr);
-    // Many 256-wide tiles: the CTA-pair kernel.
+    // 256-wide tiles filling at least half the SMs: the CTA-pair kernel
+    // (measured faster than one 128 x 256 tile per CTA from 2048 x 2048 up).
     if (K % 256 == 0 && !plan.swap && plan.splits == 1 && plan.bq == 256 && M >= 256 &&
-        plan.tiles_p * plan.tiles_q > info->num_sms && pair_kernel_enabled() && !plan_override().set)
+        2 * plan.tiles_p * plan.tiles_q >= info->num_sms && pair_kernel_enabled() && !plan_override().set)
         return pair_gemm(dev, info, A, sA, B, sB, alpha, D, M, N, K, stream);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
