@@ -37,6 +37,7 @@ struct DeviceInfo {
     int num_sms = 0;
     uint64_t smem_attr_set = 0;  // bit per kernel instantiation
     int pair_clusters = -1;      // co-resident 2-CTA clusters of the pair kernel (-1: not queried)
+    std::map<uint32_t, int> split_clusters;   // co-resident split-K clusters per (kernel, cluster size)
 };
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_devices;
@@ -192,7 +193,60 @@ PlanOverride plan_override() {
     return o;
 }
 
-Plan make_plan(int M, int N, int K, int num_sms, bool sfr) {
+// How many clusters of `splits` CTAs of a split-K instantiation fit on the
+// GPU at once (cudaOccupancyMaxActiveClusters, queried once and cached).  A
+// grid with more clusters than this runs in two waves, which for these
+// latency-bound shapes costs more than halving the split.
+template <int BQ, bool SWAP, bool SFR>
+int split_cluster_capacity(DeviceInfo* info, int splits) {
+    using C = TileConfig<BQ, true>;
+    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, true, SFR>;
+    const uint32_t key = (uint32_t)BQ | (SWAP ? 1u << 10 : 0u) | (SFR ? 1u << 11 : 0u) | ((uint32_t)splits << 12);
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = info->split_clusters.find(key);
+    if (it != info->split_clusters.end()) return it->second;
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3((unsigned)splits, 1, 1);
+        q.blockDim = dim3(nvfp4::kThreads, 1, 1);
+        q.dynamicSmemBytes = C::SMEM_BYTES;
+        cudaLaunchAttribute ca[1];
+        ca[0].id = cudaLaunchAttributeClusterDimension;
+        ca[0].val.clusterDim.x = (unsigned)splits;
+        ca[0].val.clusterDim.y = 1;
+        ca[0].val.clusterDim.z = 1;
+        q.attrs = ca;
+        q.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    info->split_clusters[key] = n;
+    return n;
+}
+
+template <bool SWAP, bool SFR>
+int split_cluster_capacity_bq(DeviceInfo* info, int bq, int splits) {
+    switch (bq) {
+        case 16: return split_cluster_capacity<16, SWAP, SFR>(info, splits);
+        case 32: return split_cluster_capacity<32, SWAP, SFR>(info, splits);
+        case 64: return split_cluster_capacity<64, SWAP, SFR>(info, splits);
+        case 128: return split_cluster_capacity<128, SWAP, SFR>(info, splits);
+        case 256: return split_cluster_capacity<256, SWAP, SFR>(info, splits);
+        default: return 0;
+    }
+}
+
+int split_cluster_capacity_of(DeviceInfo* info, bool swap, int bq, bool sfr, int splits) {
+    if (swap) return sfr ? split_cluster_capacity_bq<true, true>(info, bq, splits)
+                         : split_cluster_capacity_bq<true, false>(info, bq, splits);
+    return sfr ? split_cluster_capacity_bq<false, true>(info, bq, splits)
+               : split_cluster_capacity_bq<false, false>(info, bq, splits);
+}
+
+Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr) {
+    const int num_sms = info->num_sms;
     Plan p{};
     p.k_tiles = (K + 255) / 256;
     const PlanOverride o = plan_override();
@@ -214,18 +268,27 @@ Plan make_plan(int M, int N, int K, int num_sms, bool sfr) {
         if (!sfr && M > p.bq) p.bq = 64;   // one Q tile: scale atoms start on row 0
     } else {
         p.swap = false;
-        p.bq = M <= 256 ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
+        if (N <= 256 && M > 256)
+            p.bq = M <= 512 ? 32 : 64;   // few weight columns: more, narrower tiles
+        else
+            p.bq = M <= 256 ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
+        // Without row-major scale tiles the scales of a Q tile come as whole
+        // 128-row atoms, so a narrower Q tile is only possible alone.
+        if (!sfr && p.bq < 128 && N > p.bq) p.bq = 128;
     }
     p.tiles_p = p.swap ? (N + 127) / 128 : (M + 127) / 128;
     p.tiles_q = p.swap ? (M + p.bq - 1) / p.bq : (N + p.bq - 1) / p.bq;
     // Split K over a cluster of up to 8 CTAs (a power of two, so that the 128
     // tile rows divide evenly in the reduction) while the grid stays at or
     // below ~128 CTAs, which leaves room for the next kernel's CTAs to start
-    // (programmatic dependent launch) on the remaining SMs.
+    // (programmatic dependent launch), and all of its clusters fit on the GPU
+    // at once.  (Clusters of 16 win for one shape timed alone but lose in a
+    // sequence of different shapes: they wait for whole free GPCs.)
     const int tiles = p.tiles_p * p.tiles_q;
     const int cap = std::min(num_sms, 128);
     int splits = 1;
-    while (splits * 2 <= 8 && splits * 2 <= p.k_tiles && tiles * splits * 2 <= cap) splits *= 2;
+    for (int s = 2; s <= 8 && s <= p.k_tiles && tiles * s <= cap; s *= 2)
+        if (split_cluster_capacity_of(info, p.swap, p.bq, sfr, s) >= tiles) splits = s;
     p.splits = splits;
     return p;
 }
@@ -538,7 +601,7 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     // 16-byte aligned TMA box; otherwise they are re-laid out in global
     // scratch first.
     const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
-    const Plan plan = make_plan(M, N, K, info->num_sms, sfr);
+    const Plan plan = make_plan(M, N, K, info, sfr);
     // 256-wide tiles filling at least half the SMs: the CTA-pair kernel
     // (measured faster than one 128 x 256 tile per CTA from 2048 x 2048 up).
     if (K % 256 == 0 && !plan.swap && plan.splits == 1 && plan.bq == 256 && M >= 256 &&
@@ -753,7 +816,7 @@ nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA, const void* B, co
     if ((st = noalloc_scratch_address(dev, &scratch)) != NVFP4_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
-    const Plan plan = make_plan(M, N, K, info->num_sms, /*sfr=*/false);
+    const Plan plan = make_plan(M, N, K, info, /*sfr=*/false);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
     const void* sP = plan.swap ? sB : sA;

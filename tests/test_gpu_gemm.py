@@ -98,6 +98,8 @@ SHAPES = [
     (37, 136, 320, "moe", 24),           # K tail: 5 steps = 1 stage + 1 step
     (256, 256, 2048, "uniform", 25),
     (512, 768, 768, "normal", 26),
+    (200, 264, 320, "moe", 27),          # K tail, non-swapped: scale atoms, several Q tiles
+    (700, 256, 1024, "uniform", 28),     # few weight columns: narrow non-swapped tiles
 ]
 
 

@@ -34,6 +34,7 @@ def dev(x):
     (8, 768, 6144, "normal", 1000),    # the single attention-projection GEMM
     (300, 520, 1024, "uniform", 22),   # non-swapped tiles, ragged M and N
     (37, 136, 320, "moe", 24),         # K tail (320 = 5 MMA steps)
+    (200, 264, 512, "moe", 29),        # non-swapped, several Q tiles over scale atoms
 ])
 def test_noalloc_matches_regular_entry_point_twice(nv, M, N, K, kind, seed):
     ca, sa, cb, sb, alpha = quantized_problem(M, N, K, kind, seed)
