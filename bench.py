@@ -337,13 +337,8 @@ def load_traffic():
 
 
 def source_hash() -> str:
-    import hashlib
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "nvfp4_block_scaled_gemm_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
-    return h.hexdigest()[:16]
+    from nvfp4_block_scaled_gemm_b200.build import source_hash as h
+    return h()
 
 
 def run_e2e(nv, torch, dev, base, steps, stream):

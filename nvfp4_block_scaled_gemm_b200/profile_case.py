@@ -3,6 +3,13 @@
     python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes 512x768x6144 --iters 3
     python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes attn --iters 2
 
+`--traffic-csv FILE` (no GPU) instead turns the CSV log of an ncu run of
+`--shapes attn --iters 2` with the metrics gpu__time_duration.sum,
+dram__bytes_read.sum and dram__bytes_write.sum on the GEMM kernel into the
+per-launch DRAM summary that bench.py reports as `roofline.traffic`
+(profiles/traffic_attn_sweep.json), stamped with the hash of the kernel
+sources it was taken on.
+
 `attn` expands to the attention-projection sweep (M in {1,16,64,128,256,512},
 N=768, K=6144).  Inputs are seeded N(0,1) fp32 quantised on the GPU; every
 launch of a shape uses the same buffers (ncu flushes the caches between its
@@ -29,12 +36,65 @@ def parse_shapes(text: str):
     return out
 
 
+def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
+    """Per-launch DRAM bytes of the attention sweep from an ncu CSV log (the
+    last of the `iters` launches of each shape, in sweep order)."""
+    import csv
+    import json
+
+    from nvfp4_block_scaled_gemm_b200.build import source_hash
+
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    launches = {}
+    for row in csv.DictReader(lines):
+        if "nvfp4_gemm_kernel" not in row["Kernel Name"]:
+            continue
+        rec = launches.setdefault(int(row["ID"]), {})
+        unit = row["Metric Unit"].strip().lower()
+        val = float(row["Metric Value"].replace(",", ""))
+        scale = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "ns": 1e-3, "nsecond": 1e-3, "us": 1.0,
+                 "usecond": 1.0, "ms": 1e3, "msecond": 1e3}.get(unit, 1.0)
+        rec[row["Metric Name"]] = val * scale
+    ids = sorted(launches)
+    shapes = parse_shapes("attn")
+    if len(ids) != iters * len(shapes):
+        raise SystemExit(f"expected {iters * len(shapes)} GEMM launches in {csv_path}, found {len(ids)}")
+    per_read, per_write, per_us = {}, {}, {}
+    for i, (m, _, _) in enumerate(shapes):
+        rec = launches[ids[iters * i + iters - 1]]
+        per_read[f"M{m}"] = int(rec["dram__bytes_read.sum"])
+        per_write[f"M{m}"] = int(rec["dram__bytes_write.sum"])
+        per_us[f"M{m}"] = round(rec["gpu__time_duration.sum"], 2)
+    mean = sum(per_read[k] + per_write[k] for k in per_read) / len(per_read)
+    out = {
+        "kernel": "nvfp4_gemm_kernel",
+        "workload": "attention sweep M in {1,16,64,128,256,512}, N=768, K=6144",
+        "dram_bytes_per_launch": int(round(mean)),
+        "per_shape_dram_read": per_read,
+        "per_shape_dram_write": per_write,
+        "per_shape_us_under_ncu": per_us,
+        "source_hash": source_hash(),
+        "command": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum "
+                   "--clock-control none -k regex:nvfp4_gemm_kernel --csv --log-file traffic_attn.csv "
+                   "python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes attn --iters 2",
+    }
+    with open(out_path, "w") as f:
+        json.dump(out, f, indent=1)
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--shapes", default="512x768x6144")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--traffic-csv", default=None, help="ncu CSV of `--shapes attn --iters 2` (pass --iters 2)")
+    ap.add_argument("--traffic-out", default="profiles/traffic_attn_sweep.json")
     args = ap.parse_args()
+    if args.traffic_csv:
+        print(summarize_traffic(args.traffic_csv, args.traffic_out, args.iters))
+        return
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev)
     for (M, N, K) in parse_shapes(args.shapes):
