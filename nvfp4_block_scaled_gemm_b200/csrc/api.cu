@@ -102,6 +102,32 @@ nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** o
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Per (device, stream) pair of unit counters for the grouped kernel's
+// run-time hand-out of work units: zeroed once here, and by the last CTA of
+// every launch after that.  Launches on one stream run in order, so they
+// share it; other streams get their own.
+std::map<std::pair<int, uintptr_t>, unsigned*> g_unit_counters;
+
+nvfp4_status get_unit_counter(int dev, cudaStream_t stream, unsigned** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    unsigned*& c = g_unit_counters[{dev, reinterpret_cast<uintptr_t>(stream)}];
+    if (c == nullptr) {
+        void* p = nullptr;
+        if (cudaMalloc(&p, 2 * sizeof(unsigned)) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_NO_MEMORY;
+        }
+        if (cudaMemsetAsync(p, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) {
+            cudaGetLastError();
+            cudaFree(p);
+            return NVFP4_ERR_CUDA;
+        }
+        c = static_cast<unsigned*>(p);
+    }
+    *out = c;
+    return NVFP4_OK;
+}
+
 // ------------------------------------------------------------ tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -702,6 +728,7 @@ nvfp4_status nvfp4_grouped_gemm(const void* A, const void* sA, const void* B, co
     prm.M_total = M_total;
     prm.tiles_n = (N + 127) / 128;
     prm.k_tiles = K / 256;
+    if ((st = get_unit_counter(dev, stream, &prm.counter)) != NVFP4_OK) return st;
     auto kern = nvfp4::nvfp4_grouped_kernel;
     {
         std::lock_guard<std::mutex> lk(g_mu);

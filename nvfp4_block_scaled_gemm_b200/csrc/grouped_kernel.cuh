@@ -4,13 +4,20 @@
 // Real Inference" -- about 16 rows per expert -- and "Knowledge Created and
 // Its Impact" -- persistent grouped kernels).
 //
-// Persistent kernel.  A work unit is (expert g, 128-row tile of B[g]); CTA b
-// takes units b, b + gridDim.x, ...  The weights sit on the tensor cores'
-// 128-row M side and the expert's tokens on the N side, in passes of up to 128
-// rows; each pass loads only ceil(rows/16) 16-row boxes of A and runs MMAs
-// with N = that many rows rounded up to 16 (the instruction descriptor is
-// built at run time).  Empty experts cost two loads of row_offsets and never
-// touch their weights.
+// Persistent kernel.  A work unit is (expert g, 128-row tile of B[g]).  Units
+// are handed out at run time: each CTA's producer takes the next unit index
+// from a global counter (atomicAdd) while its current unit streams, so CTAs
+// that drew expensive units take fewer; the last CTA to finish zeroes the
+// counter for the next launch on the stream.  Unit indices run over the
+// experts with more than 128 rows (several passes) first, then the others,
+// which makes the greedy hand-out close to longest-first.  The weights sit on
+// the tensor cores' 128-row M side and the expert's tokens on the N side, in
+// passes of up to 128 rows; each pass loads only ceil(rows/16) 16-row boxes
+// of A and runs MMAs with N = that many rows rounded up to 16 (the instruction
+// descriptor is built at run time).  Empty experts are never handed out.
+//
+// The producer passes each unit to the other roles through a small ring of
+// unit descriptors in shared memory (job_full / job_empty barriers).
 //
 // Warp roles (320 threads): warp 0 TMA producer; warp 1 TMEM allocator and
 // MMA issuer; warps 2..5 epilogue (TMEM -> alpha[g] -> BF16 -> D); warps 6..9
@@ -25,6 +32,8 @@ namespace nvfp4 {
 
 constexpr int kGroupedThreads = 320;
 constexpr int kGroupedBQ = 128;   // max tokens per pass
+constexpr int kJobSlots = 4;      // unit descriptors in flight between the producer and the other roles
+constexpr int kOrderMax = 2048;   // experts ordered heavy-first in shared memory (natural order beyond)
 
 struct GroupedParams {
     const float* alpha;           // [G]
@@ -33,6 +42,7 @@ struct GroupedParams {
     int G, N, K, M_total;
     int tiles_n;                  // ceil(N / 128)
     int k_tiles;                  // K / 256
+    unsigned* counter;            // [2]: next unit, CTAs finished; zero between launches
 };
 
 struct GroupedConfig {
@@ -45,7 +55,8 @@ struct GroupedConfig {
     static constexpr int STAGES_FIT = (kSmemLimit - 2048) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
     static_assert(STAGES >= kScaleBuffers, "scale buffers are released through the ring barriers");
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
+    static constexpr int TAIL_BYTES = 1024 + 2 * kOrderMax;     // barriers, job ring, expert order
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TAIL_BYTES;
     // TMEM: two accumulators [0,BQ) and [BQ,2BQ), then 4 scale buffers of 32.
     static constexpr int ACC_COLS = BQ;
     static constexpr int SF_BASE = 2 * BQ;
@@ -55,39 +66,12 @@ struct GroupedConfig {
     static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
 };
 
-// Walks the (unit, pass) sequence of this CTA; every role advances its own
-// copy in the same order.
-struct JobCursor {
-    int unit, units, stride;
-    int g, nt, r0, rows, pass;
-    const GroupedParams* prm;
-
-    __device__ void init(const GroupedParams& p) {
-        prm = &p;
-        units = p.G * p.tiles_n;
-        stride = (int)gridDim.x;
-        unit = (int)blockIdx.x - stride;
-        pass = 0;
-        rows = 0;
-        advance_unit();
-    }
-    __device__ void advance_unit() {
-        for (unit += stride; unit < units; unit += stride) {
-            g = unit / prm->tiles_n;
-            nt = unit % prm->tiles_n;
-            r0 = __ldg(prm->offsets + g);
-            rows = __ldg(prm->offsets + g + 1) - r0;
-            if (rows > 0) break;          // empty experts: nothing to load
-        }
-        pass = 0;
-    }
-    __device__ bool valid() const { return unit < units; }
-    __device__ int q_row0() const { return r0 + pass * kGroupedBQ; }
-    __device__ int q_rows() const { return min(kGroupedBQ, rows - pass * kGroupedBQ); }
-    __device__ void next() {
-        if ((pass + 1) * kGroupedBQ < rows) ++pass;
-        else advance_unit();
-    }
+// One unit as the roles see it: expert g, weight tile nt, its token rows.
+struct UnitJob {
+    int g, nt, r0, rows;
+    __device__ int passes() const { return (rows + kGroupedBQ - 1) / kGroupedBQ; }
+    __device__ int q_row0(int pass) const { return r0 + pass * kGroupedBQ; }
+    __device__ int q_rows(int pass) const { return min(kGroupedBQ, rows - pass * kGroupedBQ); }
 };
 
 __global__ void __launch_bounds__(kGroupedThreads, 1)
@@ -99,11 +83,16 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     constexpr int NB = kScaleBuffers;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+    uint8_t* tail = smem + S * C::STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
     // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB, +2) acc_full,
-    //       [2S+NB+2, +2) acc_empty
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + NB + 4);
+    //       [2S+NB+2, +2) acc_empty, then job_full[kJobSlots], job_empty[kJobSlots]
+    constexpr int NBARS = 2 * S + NB + 4 + 2 * kJobSlots;
+    static_assert(NBARS * 8 + 8 <= 256, "tail layout");
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int4* jobs = reinterpret_cast<volatile int4*>(tail + 256);   // unit descriptors {g, nt, r0, rows}
+    int16_t* order = reinterpret_cast<int16_t*>(tail + 512);             // experts, heavy first
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t smem_base = smem_addr(smem);
@@ -113,6 +102,8 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     auto sf_ready_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
     auto acc_full_bar = [&](int a) { return bar_base + 8u * (2 * S + NB + a); };
     auto acc_empty_bar = [&](int a) { return bar_base + 8u * (2 * S + NB + 2 + a); };
+    auto job_full_bar = [&](int j) { return bar_base + 8u * (2 * S + NB + 4 + j); };
+    auto job_empty_bar = [&](int j) { return bar_base + 8u * (2 * S + NB + 4 + kJobSlots + j); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -123,6 +114,10 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(acc_full_bar(a), 1);
             mbar_init(acc_empty_bar(a), 4);
+        }
+        for (int j = 0; j < kJobSlots; ++j) {
+            mbar_init(job_full_bar(j), 1);
+            mbar_init(job_empty_bar(j), 9);   // MMA issuer, 4 writer warps, 4 epilogue warps
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -144,29 +139,93 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     grid_launch_dependents();
     grid_dependency_wait();
 
-    JobCursor job;
-    job.init(prm);
+    // Consumers take unit j from ring slot j % kJobSlots; false ends the loop
+    // (no more units, or an abort).  Lane 0 waits; the descriptor is broadcast.
+    auto take_job = [&](int j, UnitJob& jb, bool whole_warp) -> bool {
+        const int slot = j % kJobSlots;
+        int4 d = make_int4(-1, 0, 0, 0);
+        if (lane == 0 && mbar_wait(job_full_bar(slot), (uint32_t)(j / kJobSlots) & 1u, abort_flag)) {
+            d.x = jobs[slot].x;
+            d.y = jobs[slot].y;
+            d.z = jobs[slot].z;
+            d.w = jobs[slot].w;
+            mbar_arrive(job_empty_bar(slot));
+        }
+        if (whole_warp) {
+            d.x = __shfl_sync(0xffffffffu, d.x, 0);
+            d.y = __shfl_sync(0xffffffffu, d.y, 0);
+            d.z = __shfl_sync(0xffffffffu, d.z, 0);
+            d.w = __shfl_sync(0xffffffffu, d.w, 0);
+        }
+        jb.g = d.x, jb.nt = d.y, jb.r0 = d.z, jb.rows = d.w;
+        return d.x >= 0;
+    };
 
     if (warp == 0) {
+        // ---- expert order (heavy first), then the producer on lane 0
+        const bool ordered = prm.G <= kOrderMax;
+        int listed = prm.G;
+        if (ordered) {
+            listed = 0;
+            for (int heavy = 1; heavy >= 0; --heavy)
+                for (int base = 0; base < prm.G; base += 32) {
+                    const int e = base + lane;
+                    const int rows = e < prm.G ? __ldg(prm.offsets + e + 1) - __ldg(prm.offsets + e) : 0;
+                    const bool take = heavy ? rows > kGroupedBQ : (rows > 0 && rows <= kGroupedBQ);
+                    const unsigned m = __ballot_sync(0xffffffffu, take);
+                    if (take) order[listed + __popc(m & ((1u << lane) - 1u))] = (int16_t)e;
+                    listed += __popc(m);
+                }
+        }
+        __syncwarp();
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();   // each weight tile is read by one unit
             const uint64_t pol_a = policy_evict_last();    // token rows are shared by all N tiles
+            const unsigned total = (unsigned)listed * (unsigned)prm.tiles_n;
+            auto describe = [&](unsigned u, UnitJob& jb) {
+                const int idx = (int)(u / (unsigned)prm.tiles_n);
+                jb.nt = (int)(u % (unsigned)prm.tiles_n);
+                jb.g = ordered ? (int)order[idx] : idx;
+                jb.r0 = __ldg(prm.offsets + jb.g);
+                jb.rows = __ldg(prm.offsets + jb.g + 1) - jb.r0;
+            };
+            unsigned u_next = atomicAdd(prm.counter, 1u);
             int it = 0;
-            for (; job.valid(); job.next()) {
-                const int nbox = (job.q_rows() + 15) / 16;
-                const int brow = job.g * prm.N + job.nt * kBM;   // row of B viewed as [G*N][K/2]
-                for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
-                    const int s = it % S;
-                    if (!mbar_wait(empty_bar(s), ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag)) goto producer_done;
-                    const uint32_t st = smem_base + s * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + 16 * kBM + nbox * (16 * kStageKBytes + 16 * 16));
-                    tma_load_2d(st, &tmB, full_bar(s), kt * kStageKBytes, brow, pol_w);
-                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSB, full_bar(s), kt * 16, brow, pol_w);
-                    for (int bx = 0; bx < nbox; ++bx) {
-                        tma_load_2d(st + C::P_BYTES + bx * 16 * kStageKBytes, &tmA, full_bar(s), kt * kStageKBytes,
-                                    job.q_row0() + 16 * bx, pol_a);
-                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + bx * 256, &tmSA, full_bar(s),
-                                    kt * 16, job.q_row0() + 16 * bx, pol_a);
+            for (int j = 0;; ++j) {
+                UnitJob jb{-1, 0, 0, 0};
+                bool have = false;
+                for (unsigned u = u_next; u < total; u = atomicAdd(prm.counter, 1u)) {
+                    describe(u, jb);
+                    if (jb.rows > 0) {   // empty experts appear only without the order table
+                        have = true;
+                        break;
+                    }
+                }
+                if (have) u_next = atomicAdd(prm.counter, 1u);   // next index, fetched while this unit streams
+                const int slot = j % kJobSlots;
+                if (!mbar_wait(job_empty_bar(slot), ((uint32_t)(j / kJobSlots) & 1u) ^ 1u, abort_flag)) break;
+                jobs[slot].x = have ? jb.g : -1;
+                jobs[slot].y = jb.nt;
+                jobs[slot].z = jb.r0;
+                jobs[slot].w = jb.rows;
+                mbar_arrive(job_full_bar(slot));
+                if (!have) break;
+                const int brow = jb.g * prm.N + jb.nt * kBM;   // row of B viewed as [G*N][K/2]
+                for (int pass = 0; pass < jb.passes(); ++pass) {
+                    const int nbox = (jb.q_rows(pass) + 15) / 16;
+                    for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
+                        const int s = it % S;
+                        if (!mbar_wait(empty_bar(s), ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag)) goto producer_done;
+                        const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                        mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + 16 * kBM + nbox * (16 * kStageKBytes + 16 * 16));
+                        tma_load_2d(st, &tmB, full_bar(s), kt * kStageKBytes, brow, pol_w);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSB, full_bar(s), kt * 16, brow, pol_w);
+                        for (int bx = 0; bx < nbox; ++bx) {
+                            tma_load_2d(st + C::P_BYTES + bx * 16 * kStageKBytes, &tmA, full_bar(s), kt * kStageKBytes,
+                                        jb.q_row0(pass) + 16 * bx, pol_a);
+                            tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + bx * 256, &tmSA, full_bar(s),
+                                        kt * 16, jb.q_row0(pass) + 16 * bx, pol_a);
+                        }
                     }
                 }
             }
@@ -175,31 +234,37 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             int it = 0, jc = 0;
-            for (; job.valid(); job.next(), ++jc) {
-                const int acc = jc & 1;
-                const uint32_t n_mma = (uint32_t)((job.q_rows() + 15) / 16 * 16);
-                const uint32_t idesc = idesc_nvf4(kBM, (int)n_mma);
-                if (!mbar_wait(acc_empty_bar(acc), ((uint32_t)(jc >> 1) & 1u) ^ 1u, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + acc * C::ACC_COLS;
-                bool ok = true;
-                for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
-                    const int s = it % S, b = it % NB;
-                    if (!mbar_wait(sf_ready_bar(b), (uint32_t)(it / NB) & 1u, abort_flag)) {
+            bool ok = true;
+            UnitJob jb;
+            for (int j = 0; ok && take_job(j, jb, false); ++j) {
+                for (int pass = 0; ok && pass < jb.passes(); ++pass, ++jc) {
+                    const int acc = jc & 1;
+                    const uint32_t n_mma = (uint32_t)((jb.q_rows(pass) + 15) / 16 * 16);
+                    const uint32_t idesc = idesc_nvf4(kBM, (int)n_mma);
+                    if (!mbar_wait(acc_empty_bar(acc), ((uint32_t)(jc >> 1) & 1u) ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t st = smem_base + s * C::STAGE_BYTES;
-                    const uint32_t sf = tmem + C::SF_BASE + b * C::SF_STRIDE;
+                    const uint32_t d_tmem = tmem + acc * C::ACC_COLS;
+                    for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
+                        const int s = it % S, b = it % NB;
+                        if (!mbar_wait(sf_ready_bar(b), (uint32_t)(it / NB) & 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                        const uint32_t sf = tmem + C::SF_BASE + b * C::SF_STRIDE;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tc_mma_nvf4(d_tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
-                                    idesc, sf + 4 * j, sf + 16 + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
-                    tc_commit(empty_bar(s));   // frees the ring stage and scale buffer b
+                        for (int q = 0; q < 4; ++q)
+                            tc_mma_nvf4(d_tmem, desc_kmajor_sw128(st + 32 * q),
+                                        desc_kmajor_sw128(st + C::P_BYTES + 32 * q), idesc, sf + 4 * q, sf + 16 + 4 * q,
+                                        (kt > 0 || q > 0) ? 1u : 0u);
+                        tc_commit(empty_bar(s));   // frees the ring stage and scale buffer b
+                    }
+                    tc_commit(acc_full_bar(acc));
                 }
-                tc_commit(acc_full_bar(acc));
-                if (!ok) break;
             }
         }
         __syncwarp();
@@ -209,15 +274,17 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
         int it = 0;
         bool ok = true;
-        for (; ok && job.valid(); job.next()) {
-            for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
-                const int s = it % S, b = it % NB, j = it - NB;
+        UnitJob jb;
+        for (int j = 0; ok && take_job(j, jb, true); ++j) {
+            const int steps = jb.passes() * prm.k_tiles;
+            for (int u = 0; u < steps; ++u, ++it) {
+                const int s = it % S, b = it % NB, jj = it - NB;
                 int got = 1;
                 // scale buffer b was last used by K tile it - NB, released by
                 // the MMA commit on that tile's ring stage
                 if (lane == 0)
                     got = mbar_wait(full_bar(s), (uint32_t)(it / S) & 1u, abort_flag) &&
-                          (j < 0 || mbar_wait(empty_bar(j % S), (uint32_t)(j / S) & 1u, abort_flag));
+                          (jj < 0 || mbar_wait(empty_bar(jj % S), (uint32_t)(jj / S) & 1u, abort_flag));
                 if (!__shfl_sync(0xffffffffu, got, 0)) {
                     ok = false;
                     break;
@@ -240,30 +307,38 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         const int quad = warp & 3;
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
         int jc = 0;
-        for (; job.valid(); job.next(), ++jc) {
-            const int acc = jc & 1;
-            int ok = 1;
-            if (lane == 0) ok = mbar_wait(acc_full_bar(acc), (uint32_t)(jc >> 1) & 1u, abort_flag) ? 1 : 0;
-            if (!__shfl_sync(0xffffffffu, ok, 0) || *abort_flag) break;
-            tc_fence_after();
-            const int n = job.nt * kBM + quad * 32 + lane;     // output column
-            const int q0 = job.q_row0(), nq = job.q_rows();
-            const float alpha = __ldg(prm.alpha + job.g);
-#pragma unroll 1
-            for (int c0 = 0; c0 < nq; c0 += 16) {
-                uint32_t r[16];
-                tmem_load_16(t_quad + acc * C::ACC_COLS + c0, r);
-                tmem_wait_load();
-                if (n < prm.N) {
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        if (c0 + c < nq)
-                            prm.D[(size_t)(q0 + c0 + c) * prm.N + n] = __float2bfloat16_rn(__uint_as_float(r[c]) * alpha);
+        bool live = true;
+        UnitJob jb;
+        for (int j = 0; live && take_job(j, jb, true); ++j) {
+            const float alpha = __ldg(prm.alpha + jb.g);
+            const int n = jb.nt * kBM + quad * 32 + lane;     // output column
+            for (int pass = 0; pass < jb.passes(); ++pass, ++jc) {
+                const int acc = jc & 1;
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(acc_full_bar(acc), (uint32_t)(jc >> 1) & 1u, abort_flag) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, ok, 0) || *abort_flag) {
+                    live = false;
+                    break;
                 }
+                tc_fence_after();
+                const int q0 = jb.q_row0(pass), nq = jb.q_rows(pass);
+#pragma unroll 1
+                for (int c0 = 0; c0 < nq; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_load_16(t_quad + acc * C::ACC_COLS + c0, r);
+                    tmem_wait_load();
+                    if (n < prm.N) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            if (c0 + c < nq)
+                                prm.D[(size_t)(q0 + c0 + c) * prm.N + n] =
+                                    __float2bfloat16_rn(__uint_as_float(r[c]) * alpha);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty_bar(acc));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty_bar(acc));
         }
     }
 
@@ -272,6 +347,16 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    // The last CTA to finish zeroes the unit counter for the next launch (no
+    // CTA fetches after it has counted itself finished).
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(prm.counter + 1, 1u) == gridDim.x - 1) {
+            atomicExch(prm.counter, 0u);
+            atomicExch(prm.counter + 1, 0u);
+            __threadfence();
+        }
     }
 }
 

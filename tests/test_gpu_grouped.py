@@ -93,3 +93,59 @@ def test_grouped_full_size_sampled(nv):
         sel = group == g
         _, ref, ad = oracle.gemm_sampled(A, sA, B[g], sB[g], float(alpha[g]), Mt, N, K, rows[sel], cols[sel])
         assert not violations(got[rows[sel], cols[sel]], ref, ad).any(), f"expert {g}"
+
+
+def test_grouped_repeated_launches_on_two_streams(nv):
+    # Work units are handed out at run time from a per-stream counter that the
+    # last CTA of each launch zeroes: back-to-back launches on one stream and
+    # launches on a second stream must each cover every unit exactly once.
+    rng = np.random.default_rng(5)
+    G, N, K = 9, 392, 768
+    counts = [0, 260, 5, 0, 129, 1, 0, 77, 16]
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    Mt = int(off[-1])
+    A = synth.random_codes(Mt, K, 31)
+    sA = synth.random_scales(Mt, K, 32)
+    B = np.stack([synth.random_codes(N, K, 40 + g) for g in range(G)])
+    sB = np.stack([synth.random_scales(N, K, 50 + g) for g in range(G)])
+    alpha = rng.uniform(0.5, 2.0, G).astype(np.float32)
+    _, ref, ad = oracle.grouped_gemm(A, sA, B, sB, alpha, off, G, Mt, N, K)
+    args = [dev(A), dev(sA), dev(B), dev(sB), dev(alpha), dev(off)]
+    other = torch.cuda.Stream()
+    outs = []
+    for s in (None, None, None, other, other):
+        D = torch.full((Mt, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        if s is other:
+            other.wait_stream(torch.cuda.current_stream())   # inputs and the NaN fill come first
+            with torch.cuda.stream(other):
+                nv.grouped_gemm(*args, out=D, stream=other)
+        else:
+            nv.grouped_gemm(*args, out=D)
+        outs.append(D)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    first = outs[0].view(torch.int16)
+    for D in outs:
+        assert torch.equal(D.view(torch.int16), first)     # one CTA computes each unit: bit-identical
+    assert not violations(outs[0].float().cpu().numpy(), ref, ad).any()
+
+
+def test_grouped_more_experts_than_the_order_table(nv):
+    # More than 2048 experts: units are handed out in expert order instead of
+    # heavy experts first, skipping the empty ones at run time.
+    rng = np.random.default_rng(6)
+    G, N, K = 2100, 128, 256
+    counts = np.zeros(G, np.int64)
+    hot = rng.choice(G, 40, replace=False)
+    counts[hot] = rng.integers(1, 40, 40)
+    counts[hot[0]] = 200                     # one expert over a 128-row pass
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    Mt = int(off[-1])
+    A = synth.random_codes(Mt, K, 61)
+    sA = synth.random_scales(Mt, K, 62)
+    B = synth.random_codes(G * N, K, 63).reshape(G, N, K // 2)
+    sB = synth.random_scales(G * N, K, 64).reshape(G, N, K // 16)
+    alpha = rng.uniform(0.5, 2.0, G).astype(np.float32)
+    _, ref, ad = oracle.grouped_gemm(A, sA, B, sB, alpha, off, G, Mt, N, K)
+    got = run(nv, A, sA, B, sB, alpha, off)
+    assert not violations(got, ref, ad).any()
