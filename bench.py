@@ -452,6 +452,27 @@ def time_single_shape(nv, torch, dev, M, Nn, Kk, kind, seed, iters, stream, b_co
     return e0.elapsed_time(e1) * 1e3 / (reps * R)
 
 
+def measure_fp4_peak(nv, torch, stream, steps=200000, reps=3):
+    """Dense FP4 tensor-core rate from the library's calibration kernel
+    (back-to-back block-scaled MMAs on resident operands): TFLOP/s for the
+    1-CTA and the 2-CTA (CTA pair) instruction forms."""
+    out = {}
+    for pair in (False, True):
+        with torch.cuda.stream(stream):
+            nv.fp4_peak_probe(pair, steps // 10, stream)          # warm-up
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ctas = 0
+            for _ in range(reps):
+                ctas = nv.fp4_peak_probe(pair, steps, stream)
+            e1.record(stream)
+        stream.synchronize()
+        assert nv.get_device_error(stream) == 0
+        secs = e0.elapsed_time(e1) / 1e3 / reps
+        out["cta_pair" if pair else "one_cta"] = round(steps * ctas * nv.FP4_PEAK_FLOPS_PER_STEP / secs / 1e12, 1)
+    return out
+
+
 def run_shapes(args, shapes, label):
     import torch
     import nvfp4_block_scaled_gemm_b200 as nv
@@ -460,16 +481,24 @@ def run_shapes(args, shapes, label):
     hbm_gbs, bf16_tf, src = load_peaks()
     fp4_tf = 4.0 * bf16_tf      # dense FP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
     stream = torch.cuda.Stream()
+    calib = measure_fp4_peak(nv, torch, stream) if label == "saturation" else None
     rows = []
     for (name, M, Nn, Kk, kind, seed) in shapes:
         us = time_single_shape(nv, torch, dev, M, Nn, Kk, kind, seed, args.steps, stream)
         b, f = accounting.gemm_bytes(M, Nn, Kk), accounting.gemm_flops(M, Nn, Kk)
         t_roof = max(b / (hbm_gbs * 1e9), f / (fp4_tf * 1e12))
-        rows.append({"name": name, "M": M, "N": Nn, "K": Kk, "us": round(us, 2), "GBps": round(b / us / 1e3, 1),
-                     "TFLOPS": round(f / us / 1e6, 1), "roofline_frac": round(t_roof / (us * 1e-6), 4),
-                     "bound": "hbm" if b / (hbm_gbs * 1e9) >= f / (fp4_tf * 1e12) else "tensor"})
-    return {"workload": label, "peaks": {"hbm_gbs": hbm_gbs, "fp4_tflops": fp4_tf, "source": f"{src} (fp4 = 4 x bf16)"},
-            "shapes": rows}
+        row = {"name": name, "M": M, "N": Nn, "K": Kk, "us": round(us, 2), "GBps": round(b / us / 1e3, 1),
+               "TFLOPS": round(f / us / 1e6, 1), "roofline_frac": round(t_roof / (us * 1e-6), 4),
+               "bound": "hbm" if b / (hbm_gbs * 1e9) >= f / (fp4_tf * 1e12) else "tensor"}
+        if calib:
+            row["frac_of_calibrated_fp4"] = round(f / us / 1e6 / max(calib.values()), 4)
+            row["frac_of_nominal_9pf"] = round(f / us / 1e6 / 9000.0, 4)
+        rows.append(row)
+    peaks = {"hbm_gbs": hbm_gbs, "fp4_tflops": fp4_tf, "source": f"{src} (fp4 = 4 x bf16)"}
+    if calib:
+        peaks["fp4_calibrated_tflops"] = calib
+        peaks["fp4_nominal_tflops"] = 9000.0
+    return {"workload": label, "peaks": peaks, "shapes": rows}
 
 
 def run_grouped(args):

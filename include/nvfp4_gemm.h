@@ -180,6 +180,21 @@ const char* nvfp4_status_string(nvfp4_status status);
 nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
 /*
+ * nvfp4_fp4_peak_probe -- calibration of the dense FP4 tensor-core rate (no
+ * counterpart on the pages, which quote only a vendor-style peak for another
+ * GPU, "Peeling the Kernel Onion", section "The Results").  Launches one CTA
+ * per SM (pair = 0: tcgen05.mma.cta_group::1, 128 x 256 x 64 per instruction)
+ * or one 2-CTA cluster per two SMs (pair = 1: cta_group::2, 256 x 256 x 64 per
+ * instruction per pair), each issuing `steps` (1 .. 1e8) block-scaled
+ * kind::mxf4nvf4 MMAs back to back on operands resident in shared memory and
+ * scales resident in TMEM.  Writes the number of CTAs launched to *ctas_out.
+ * The caller times the launch on `stream`; the work is
+ * steps x ctas x 2 x 128 x 256 x 64 FLOPs in both forms.  The MMA results are
+ * discarded.  Returns NVFP4_ERR_INVALID_ARG for arguments out of range.
+ */
+nvfp4_status nvfp4_fp4_peak_probe(int pair, long long steps, int* ctas_out, void* stream);
+
+/*
  * nvfp4_gemm_noalloc -- the same GEMM as nvfp4_gemm (same arguments, layouts,
  * requirements and result), for callers that are not allowed to allocate
  * device memory during the call: runtimes that own and pool all device

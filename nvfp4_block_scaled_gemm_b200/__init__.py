@@ -32,7 +32,7 @@ EXPORTS = (
     "nvfp4_gemm", "nvfp4_gemm_ex", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
-    "nvfp4_gemm_noalloc",
+    "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe",
 )
 
 
@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_kernel_launches.restype = ctypes.c_ulonglong
         L.nvfp4_gemm_noalloc.argtypes = [P, P, P, P, f32, P, i32, i32, i32, P]
         L.nvfp4_gemm_noalloc.restype = i32
+        L.nvfp4_fp4_peak_probe.argtypes = [i32, ctypes.c_longlong, ctypes.POINTER(i32), P]
+        L.nvfp4_fp4_peak_probe.restype = i32
         _lib = L
     return _lib
 
@@ -187,6 +189,19 @@ def grouped_gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.T
                                     row_offsets.data_ptr(), G, out.data_ptr(), Mt, N, K, _stream(stream)),
            "nvfp4_grouped_gemm")
     return out
+
+
+def fp4_peak_probe(pair: bool, steps: int, stream=None) -> int:
+    """Launch the dense-FP4 calibration kernel (nvfp4_fp4_peak_probe) on
+    `stream`; returns the number of CTAs.  The launch performs
+    steps x CTAs x 2 x 128 x 256 x 64 FLOPs; time it with CUDA events."""
+    ctas = ctypes.c_int(0)
+    _check(lib().nvfp4_fp4_peak_probe(1 if pair else 0, int(steps), ctypes.byref(ctas), _stream(stream)),
+           "nvfp4_fp4_peak_probe")
+    return ctas.value
+
+
+FP4_PEAK_FLOPS_PER_STEP = 2 * 128 * 256 * 64   # per CTA and step, both forms
 
 
 def quantize(X: torch.Tensor, stream=None):

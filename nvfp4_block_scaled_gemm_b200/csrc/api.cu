@@ -18,6 +18,7 @@
 #include "gemm_kernel.cuh"
 #include "grouped_kernel.cuh"
 #include "pair_kernel.cuh"
+#include "peak_kernel.cuh"
 #include "persistent_kernel.cuh"
 
 namespace {
@@ -782,6 +783,48 @@ nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream_) {
     nvfp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>(timeout_ns);
     g_launches++;
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_fp4_peak_probe(int pair, long long steps, int* ctas_out, void* stream_) {
+    if ((pair != 0 && pair != 1) || steps < 1 || steps > 100000000ll || !ctas_out) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    auto kern = pair ? nvfp4::fp4_peak_kernel<true> : nvfp4::fp4_peak_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, nvfp4::kPeakSmem) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(nvfp4::kPeakThreads, 1, 1);
+    cfg.dynamicSmemBytes = nvfp4::kPeakSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    int ctas = info->num_sms;
+    if (pair) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(2, 1, 1);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        ctas = 2 * std::min(n, info->num_sms / 2);
+    }
+    cfg.gridDim = dim3((unsigned)ctas, 1, 1);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, steps);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    *ctas_out = ctas;
+    return NVFP4_OK;
 }
 
 }  // extern "C"

@@ -323,6 +323,8 @@ def boundary_samples(M, N, seed, n_random=4000, edge=256):
                                   # whose second half lies wholly past M (rows) and N (columns)
     (4096, 4096, 1024, False),    # 32 x 16 = 512 tiles, several tiles per CTA (pair)
     (2304, 4352, 2048, False),    # 9 x 17 pair tiles, long K
+    (1025, 4352, 256, False),     # one K tile per tile; the last tile row holds a single row of A
+    (1280, 9000, 768, False),     # last tile column holds 40 columns: the second CTA's B rows all past N
 ])
 def test_gemm_persistent_path_matches_oracle(nv, monkeypatch, pair, M, N, K, full):
     # NVFP4_GEMM_PAIR=0 selects the single-CTA persistent kernel where the
