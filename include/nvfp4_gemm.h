@@ -180,6 +180,28 @@ const char* nvfp4_status_string(nvfp4_status status);
 nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
 /*
+ * nvfp4_quantize_scaled -- quantize-and-pack with the global scale given:
+ * the activation-side step that feeds the GEMM in decode, where a tensor's
+ * global scale is fixed in advance rather than taken from its own amax
+ * ("Peeling the Kernel Onion", section "The Critical Connection to Real
+ * Inference": activations are quantized upstream of each GEMM).
+ *   X       rows x K values, row-major: fp32 (x_is_bf16 = 0) or BF16
+ *           (x_is_bf16 = 1); 16-byte aligned.  K a multiple of 16.
+ *   g       global scale, positive and finite.
+ *   codes   out: packed E2M1 [rows][K/2] (8-byte aligned), low nibble = even k.
+ *   scales  out: E4M3 block scales [rows][K/16], s = E4M3(amax_blk / (6 g))
+ *           round-to-nearest-even with saturation to 448; codes are
+ *           E2M1(x / (g * s)) with the same rounding and saturation to 6.
+ * Bit-exact with nvfp4_quantize's block steps for the same g (one launch
+ * instead of three: no amax pass).  Launched with programmatic dependent
+ * launch, so a following nvfp4_gemm on the stream starts its prologue while
+ * this kernel runs.  Returns NVFP4_ERR_INVALID_ARG for bad pointers, g <= 0
+ * or non-finite, NVFP4_ERR_UNSUPPORTED_SHAPE for K % 16 != 0.
+ */
+nvfp4_status nvfp4_quantize_scaled(const void* X, int x_is_bf16, int rows, int K, float g, void* codes,
+                                   void* scales, void* stream);
+
+/*
  * nvfp4_fp4_peak_probe -- calibration of the dense FP4 tensor-core rate (no
  * counterpart on the pages, which quote only a vendor-style peak for another
  * GPU, "Peeling the Kernel Onion", section "The Results").  Launches one CTA

@@ -32,7 +32,7 @@ EXPORTS = (
     "nvfp4_gemm", "nvfp4_gemm_ex", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
-    "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe",
+    "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe", "nvfp4_quantize_scaled",
 )
 
 
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_gemm_noalloc.restype = i32
         L.nvfp4_fp4_peak_probe.argtypes = [i32, ctypes.c_longlong, ctypes.POINTER(i32), P]
         L.nvfp4_fp4_peak_probe.restype = i32
+        L.nvfp4_quantize_scaled.argtypes = [P, i32, i32, i32, f32, P, P, P]
+        L.nvfp4_quantize_scaled.restype = i32
         _lib = L
     return _lib
 
@@ -189,6 +191,23 @@ def grouped_gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.T
                                     row_offsets.data_ptr(), G, out.data_ptr(), Mt, N, K, _stream(stream)),
            "nvfp4_grouped_gemm")
     return out
+
+
+def quantize_scaled(X: torch.Tensor, g: float, stream=None):
+    """fp32 or BF16 [rows, K] (CUDA) with a given global scale g ->
+    (codes uint8 [rows, K/2], scales uint8 [rows, K/16]) in one launch."""
+    if X.dim() != 2:
+        raise ValueError("X must be 2-D [rows, K]")
+    if X.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"X must be float32 or bfloat16, got {X.dtype}")
+    rows, K = X.shape
+    _need(X, "X", X.dtype, (rows, K))
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((rows, K // 16), dtype=torch.uint8, device=X.device)
+    _check(lib().nvfp4_quantize_scaled(X.data_ptr(), 1 if X.dtype == torch.bfloat16 else 0, rows, K, float(g),
+                                       codes.data_ptr(), scales.data_ptr(), _stream(stream)),
+           "nvfp4_quantize_scaled")
+    return codes, scales
 
 
 def fp4_peak_probe(pair: bool, steps: int, stream=None) -> int:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <atomic>
@@ -783,6 +784,41 @@ nvfp4_status nvfp4_debug_wait_timeout(uint64_t timeout_ns, void* stream_) {
     nvfp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>(timeout_ns);
     g_launches++;
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_quantize_scaled(const void* X, int x_is_bf16, int rows, int K, float g, void* codes,
+                                   void* scales, void* stream_) {
+    if (rows < 0 || K <= 0 || (x_is_bf16 != 0 && x_is_bf16 != 1)) return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!(g > 0.0f) || !std::isfinite(g)) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0) return NVFP4_OK;
+    if (!X || !codes || !scales || !aligned(X, 16) || !aligned(codes, 8)) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    const long long nb = (long long)rows * (K / 16);
+    const int threads = 256;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((nb + threads - 1) / threads), 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.stream = static_cast<cudaStream_t>(stream_);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e =
+        x_is_bf16 ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_scaled_kernel<true>, X, nb, g, static_cast<uint8_t*>(codes),
+                                       static_cast<uint8_t*>(scales))
+                  : cudaLaunchKernelEx(&cfg, nvfp4::quantize_scaled_kernel<false>, X, nb, g,
+                                       static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_fp4_peak_probe(int pair, long long steps, int* ctas_out, void* stream_) {

@@ -169,6 +169,60 @@ __global__ void quantize_kernel(const float* __restrict__ X, long long blocks, c
     scales[b] = (uint8_t)s;
 }
 
+// One pass with the global scale g given (a scale fixed in advance for the
+// activation tensor): the same block steps as quantize_kernel, on fp32 or
+// BF16 input (BF16 widens to fp32 exactly).  Launched with programmatic
+// dependent launch: it lets the next kernel (the GEMM) start its prologue at
+// once and waits for the previous kernel before reading X.
+template <bool BF16>
+__global__ void quantize_scaled_kernel(const void* __restrict__ X, long long blocks, float g,
+                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= blocks) return;
+    const float six_g = __fmul_rn(6.0f, g);
+    float x[16];
+    if (BF16) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(X) + b * 16);   // BF16 bits
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint4 v = __ldg(src + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                x[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                x[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        }
+    } else {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(X) + b * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 f = __ldg(src + i);
+            x[4 * i] = f.x;
+            x[4 * i + 1] = f.y;
+            x[4 * i + 2] = f.z;
+            x[4 * i + 3] = f.w;
+        }
+    }
+    float amax_blk = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax_blk = fmaxf(amax_blk, fabsf(x[i]));
+    const uint32_t s = e4m3_from_float(__fdiv_rn(amax_blk, six_g));
+    const float denom = __fmul_rn(g, e4m3_to_float(s));
+    uint32_t out[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = denom == 0.0f ? x[8 * h + i] * 0.0f : __fdiv_rn(x[8 * h + i], denom);
+        out[h] = e2m1x8_from_float(v);
+    }
+    *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(out[0], out[1]);
+    scales[b] = (uint8_t)s;
+}
+
 // Pass 3: replace the amax bits by the global scale g.
 __global__ void finalize_global_scale_kernel(float* g_inout) {
     g_inout[0] = global_scale_from_amax(__uint_as_float(*reinterpret_cast<unsigned*>(g_inout)));

@@ -51,6 +51,8 @@ def lib():
         L.oracle_e2m1_rne_satfinite.argtypes = [f32]
         L.oracle_quantize.restype = i32
         L.oracle_quantize.argtypes = [P, i32, i32, P, P, P]
+        L.oracle_quantize_with_scale.argtypes = [P, i32, i32, f32, P, P]
+        L.oracle_quantize_with_scale.restype = i32
         L.oracle_gemm.restype = i32
         L.oracle_gemm.argtypes = [P, P, P, P, f32, i32, i32, i32, P, P, P]
         L.oracle_gemm_sampled.restype = i32
@@ -101,6 +103,18 @@ def quantize(X: np.ndarray):
     if rc:
         raise ValueError("oracle_quantize rejected its input")
     return codes, scales, float(g[0])
+
+
+def quantize_with_scale(X: np.ndarray, g: float):
+    """fp32 [rows, K] and a given global scale g -> (codes u8 [rows, K/2], scales u8 [rows, K/16])."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    rows, K = X.shape
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((rows, K // 16), np.uint8)
+    rc = lib().oracle_quantize_with_scale(_p(X), rows, K, ctypes.c_float(g), _p(codes), _p(scales))
+    if rc:
+        raise ValueError("oracle_quantize_with_scale rejected its input")
+    return codes, scales
 
 
 def gemm(A, sA, B, sB, alpha: float, M: int, N: int, K: int):

@@ -101,17 +101,11 @@ int oracle_e2m1_rne_satfinite(float v) {
  * s = E4M3_rne_satfinite(amax_blk / (6 * g)); each element
  * q = E2M1_rne_satfinite(x / (g * decode(s))), packed two per byte with the
  * even-k element in the low nibble.  All arithmetic in IEEE fp32. */
-int oracle_quantize(const float* X, int rows, int K,
-                    uint8_t* codes, uint8_t* scales, float* g_out) {
-    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
-    float amax = 0.0f;
-    for (long i = 0; i < (long)rows * K; i++) {
-        if (!isfinite(X[i])) return -1;
-        float a = fabsf(X[i]);
-        if (a > amax) amax = a;
-    }
-    /* An all-zero tensor has no scale to recover; g = 1 keeps every step finite. */
-    volatile float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+/* The per-block steps of the quantizer for a given global scale g: block
+ * scale s = E4M3(amax_blk / (6 g)), codes = E2M1(x / (g * E4M3(s))), both
+ * round-to-nearest-even with saturation, fp32 IEEE arithmetic. */
+static void quantize_blocks(const float* X, int rows, int K, float g_in, uint8_t* codes, uint8_t* scales) {
+    volatile float g = g_in;
     volatile float six_g = 6.0f * g;
     for (int r = 0; r < rows; r++) {
         const float* x = X + (long)r * K;
@@ -141,7 +135,31 @@ int oracle_quantize(const float* X, int rows, int K,
             }
         }
     }
+}
+
+int oracle_quantize(const float* X, int rows, int K,
+                    uint8_t* codes, uint8_t* scales, float* g_out) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
+    float amax = 0.0f;
+    for (long i = 0; i < (long)rows * K; i++) {
+        if (!isfinite(X[i])) return -1;
+        float a = fabsf(X[i]);
+        if (a > amax) amax = a;
+    }
+    /* An all-zero tensor has no scale to recover; g = 1 keeps every step finite. */
+    volatile float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    quantize_blocks(X, rows, K, g, codes, scales);
     *g_out = g;
+    return 0;
+}
+
+int oracle_quantize_with_scale(const float* X, int rows, int K, float g,
+                               uint8_t* codes, uint8_t* scales) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
+    if (!(g > 0.0f) || !isfinite(g)) return -1;
+    for (long i = 0; i < (long)rows * K; i++)
+        if (!isfinite(X[i])) return -1;
+    quantize_blocks(X, rows, K, g, codes, scales);
     return 0;
 }
 

@@ -45,6 +45,14 @@ int    oracle_e2m1_rne_satfinite(float v);   /* nearest E2M1, ties to even, |v|>
 int oracle_quantize(const float* X, int rows, int K,
                     uint8_t* codes, uint8_t* scales, float* g_out);
 
+/* The same block steps with the global scale g given by the caller (a scale
+ * fixed in advance for a tensor, instead of one computed from its amax): the
+ * configs' recipe after its first step.  Block scales that would exceed 448
+ * saturate, and so do codes beyond 6.  Returns -1 for g not positive and
+ * finite or a NaN/Inf input. */
+int oracle_quantize_with_scale(const float* X, int rows, int K, float g,
+                               uint8_t* codes, uint8_t* scales);
+
 /* Exact value of one output: sets *exact (double rounding of the exact
  * value), *absdot = |alpha| * sum_k |a_k b_k| (fp64) and returns the BF16 bits
  * of the single RNE rounding of the exact value. */

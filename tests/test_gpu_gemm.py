@@ -49,6 +49,58 @@ def test_quantize_bitexact(nv, rows, K, kind, seed):
     assert (gc.cpu().numpy() == c).all()
 
 
+@pytest.mark.parametrize("bf16", [False, True])
+@pytest.mark.parametrize("rows,K,kind,seed,gmul", [
+    (8, 6144, "normal", 1000, 1.0),      # g from the tensor's own amax
+    (33, 512, "moe", 7, 0.37),           # smaller g: scales and codes saturate on outlier blocks
+    (17, 256, "uniform", 3, 5.0),        # larger g: small block scales, subnormal E4M3 bytes
+    (3, 8192, "normal", 13, 1.0)])
+def test_quantize_scaled_bitexact(nv, bf16, rows, K, kind, seed, gmul):
+    # One-launch quantizer with the global scale given, fp32 and BF16 input;
+    # BF16 values widen to fp32 exactly, so the oracle sees the same numbers.
+    X = synth.source(kind, rows, 8, K, seed)[0]
+    Xt = dev(X)
+    if bf16:
+        Xt = Xt.to(torch.bfloat16)
+        X = Xt.float().cpu().numpy()
+    g = float(np.float32(oracle.quantize(X)[2] * gmul))
+    c, s = oracle.quantize_with_scale(X, g)
+    gc, gs = nv.quantize_scaled(Xt, g)
+    torch.cuda.synchronize()
+    assert (gs.cpu().numpy() == s).all()
+    assert (gc.cpu().numpy() == c).all()
+
+
+def test_quantize_scaled_then_gemm_chain(nv):
+    # Activations quantized by nvfp4_quantize_scaled and consumed by the GEMM
+    # that follows on the stream (programmatic dependent launch between them),
+    # three times back to back with new activations each time.
+    M, N, K = 16, 768, 2048
+    W = synth.source("moe", M, N, K, 1201)[1]
+    cb, sb, gb = oracle.quantize(W)
+    B, SB = dev(cb), dev(sb)
+    for rep in range(3):
+        X = synth.activations_with_outliers(M, K, 300 + rep)
+        ga = float(np.float32(oracle.quantize(X)[2]))
+        ca, sa = oracle.quantize_with_scale(X, ga)
+        alpha = float(np.float32(ga) * np.float32(gb))
+        _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+        qa, qs = nv.quantize_scaled(dev(X), ga)
+        D = nv.gemm(qa, qs, B, SB, alpha)
+        torch.cuda.synchronize()
+        assert nv.get_device_error() == 0
+        assert not violations(D.float().cpu().numpy(), ref, ad).any()
+
+
+def test_quantize_scaled_rejects_bad_arguments(nv):
+    X = torch.ones((4, 32), device="cuda")
+    for g in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(nv.Nvfp4Error):
+            nv.quantize_scaled(X, g)
+    with pytest.raises(TypeError):
+        nv.quantize_scaled(X.half(), 1.0)
+
+
 def test_quantize_rounding_edges_bitexact(nv):
     # Values placed on E2M1 midpoints, E4M3 midpoints, zeros of both signs,
     # tiny magnitudes and saturating blocks, to pin the hardware conversions

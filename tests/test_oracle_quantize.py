@@ -137,3 +137,47 @@ def test_quantized_gemm_tracks_fp32_gemm():
     exact = A.astype(np.float64) @ B.astype(np.float64).T
     assert np.linalg.norm(ref - exact) / np.linalg.norm(exact) < 0.2
     assert np.corrcoef(ref.ravel(), exact.ravel())[0, 1] > 0.98
+
+
+# ------------------------------------------------------ given global scale
+# The configs' recipe after its first step (g fixed in advance).  Pinned to
+# the amax-scaled quantizer above, to closed forms, and to saturation.
+
+@pytest.mark.parametrize("kind,seed", [("normal", 3), ("moe", 4), ("uniform", 5)])
+def test_given_scale_equals_amax_scale_quantizer(kind, seed):
+    X = synth.source(kind, 13, 8, 96, seed)[0]
+    c, s, g = oracle.quantize(X)
+    c2, s2 = oracle.quantize_with_scale(X, g)
+    assert np.array_equal(c, c2) and np.array_equal(s, s2)
+
+
+def test_given_scale_closed_form_block():
+    # g = 1 and a block whose largest magnitude is 6: t = 6 / 6 = 1 -> E4M3 byte
+    # 0x38 (1.0), and every value on the E2M1 grid keeps its code.
+    vals = np.array([6, -3, 1.5, -0.5, 0, 4, -6, 2, 1, -1, 0.5, 3, -4, -2, -1.5, 0], np.float32)
+    codes, scales = oracle.quantize_with_scale(vals.reshape(1, 16), 1.0)
+    assert scales[0, 0] == 0x38
+    mag = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}
+    want = [(8 if v < 0 or (v == 0 and np.signbit(v)) else 0) | mag[abs(float(v))] for v in vals]
+    got = [(codes[0, k // 2] >> (4 * (k & 1))) & 0xF for k in range(16)]
+    assert got == want
+
+
+def test_given_scale_saturates():
+    # g far below amax / 2688: the block scale saturates at 448 (byte 0x7E) and
+    # values beyond 6 * 448 * g saturate to the code of +-6.
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0], x[0, 1], x[0, 2] = 1000.0, -1000.0, 0.25
+    g = 0.01
+    codes, scales = oracle.quantize_with_scale(x, g)
+    assert scales[0, 0] == 0x7E
+    c0, c1 = codes[0, 0] & 0xF, codes[0, 0] >> 4
+    assert c0 == 0x7 and c1 == 0xF            # +6 and -6
+    # 0.25 / (0.01 * 448) = 0.0558 -> nearest E2M1 is 0
+    assert codes[0, 1] & 0xF == 0
+
+
+@pytest.mark.parametrize("g", [0.0, -1.0, float("inf"), float("nan")])
+def test_given_scale_rejects_bad_scale(g):
+    with pytest.raises(ValueError):
+        oracle.quantize_with_scale(np.ones((1, 16), np.float32), g)
