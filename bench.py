@@ -549,6 +549,79 @@ def run_grouped(args):
             "note": "weights stream once per launch (1.8 GB >> L2); eager launches, events"}
 
 
+def run_chain(args, layers=8):
+    """A dependent layer sequence: attention-projection GEMMs alternating
+    M x 768 x 6144 and M x 6144 x 768 (the tensor-parallel in/out projection
+    shapes of one GPU), each layer's BF16 output quantized by
+    nvfp4_quantize_scaled with a global scale fixed from one eager calibration
+    pass, and fed to the next GEMM.  The whole chain is one CUDA graph; every
+    launch in it uses programmatic dependent launch.  Reports the time per
+    layer (quantize + GEMM) for each M."""
+    import torch
+    import nvfp4_block_scaled_gemm_b200 as nv
+    dev = torch.device("cuda", 0)
+    nv.lib()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1500)
+    dims = [(N, K), (K, N)]
+    weights = []
+    for li in range(layers):
+        n_out, k_in = dims[li % 2]
+        W = torch.randn((n_out, k_in), generator=gen, device=dev) * 0.02
+        cb, sb, gb = nv.quantize(W)
+        weights.append((cb, sb, float(gb.item())))
+    stream = torch.cuda.Stream()
+    out = []
+    for m in (1, 16, 64, 256):
+        X = torch.randn((m, K), generator=gen, device=dev).to(torch.bfloat16)
+        # calibration: amax-scaled quantization of each layer's input, once
+        g_act, cur = [], X
+        for li in range(layers):
+            cq, sq, gq = nv.quantize(cur.float())
+            g = float(gq.item())
+            g_act.append(g)
+            cb, sb, gb = weights[li]
+            cur = nv.gemm(cq, sq, cb, sb, g * gb)
+        torch.cuda.synchronize()
+        bufs = [torch.empty((m, dims[li % 2][0]), dtype=torch.bfloat16, device=dev) for li in range(layers)]
+
+        def enqueue():
+            a = X
+            for li in range(layers):
+                cq, sq = nv.quantize_scaled(a, g_act[li], stream=stream)
+                cb, sb, gb = weights[li]
+                nv.gemm(cq, sq, cb, sb, g_act[li] * gb, out=bufs[li], stream=stream)
+                a = bufs[li]
+
+        with torch.cuda.stream(stream):
+            enqueue()
+        stream.synchronize()
+        g_chain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_chain, stream=stream):
+            enqueue()
+        reps = max(3, min(args.steps, 200))
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g_chain.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g_chain.replay()
+            e1.record(stream)
+        stream.synchronize()
+        assert nv.get_device_error(stream) == 0
+        us_layer = e0.elapsed_time(e1) * 1e3 / (reps * layers)
+        b = sum(accounting.gemm_bytes(m, dims[li % 2][0], dims[li % 2][1]) for li in range(layers)) / layers
+        out.append({"M": m, "us_per_layer": round(us_layer, 2), "GBps": round(b / us_layer / 1e3, 1)})
+    return {"workload": f"dependent chain of {layers} layers (quantize_scaled + GEMM), shapes alternating "
+                        f"Mx{N}x{K} and Mx{K}x{N}, one CUDA graph, programmatic dependent launch",
+            "layers": layers, "per_M": out,
+            "note": "weights 6.3 MB per layer stay in L2 across replays (the chain is launch- and "
+                    "latency-bound, which is what it measures)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -556,7 +629,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped"], default="attn",
+    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain"], default="attn",
                     help="attn (default) prints the benchmark line; the others print a per-shape report")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -574,6 +647,8 @@ def main():
         if rank == 0:
             if args.workload == "grouped":
                 print(json.dumps(run_grouped(args)), flush=True)
+            elif args.workload == "chain":
+                print(json.dumps(run_chain(args)), flush=True)
             else:
                 shapes = synth.moe_sweep() if args.workload == "moe" else synth.saturation_sweep()
                 print(json.dumps(run_shapes(args, shapes, args.workload)), flush=True)
