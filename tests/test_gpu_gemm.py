@@ -205,7 +205,7 @@ def test_gemm_alpha_is_applied(nv):
     assert (g2 == (g1 * 0.5)).all()      # scaling by a power of two is exact in bf16 here
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 768, 6144), (256, 768, 6144), (2048, 2048, 512)])
+@pytest.mark.parametrize("M,N,K", [(1, 768, 6144), (256, 768, 6144), (2048, 2048, 512), (2048, 2048, 6144)])
 def test_gemm_deterministic(nv, M, N, K):
     ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "normal", 41)
     A, SA, B, SB = dev(ca), dev(sa), dev(cb), dev(sb)
@@ -377,6 +377,8 @@ def boundary_samples(M, N, seed, n_random=4000, edge=256):
     (2304, 4352, 2048, False),    # 9 x 17 pair tiles, long K
     (1025, 4352, 256, False),     # one K tile per tile; the last tile row holds a single row of A
     (1280, 9000, 768, False),     # last tile column holds 40 columns: the second CTA's B rows all past N
+    (2048, 2048, 6144, False),    # 64 tiles on 74 pairs: every tile cut by K between pairs (stream-K)
+    (1800, 1544, 2048, False),    # stream-K with ragged M and N (8 valid columns in the last tile column)
 ])
 def test_gemm_persistent_path_matches_oracle(nv, monkeypatch, pair, M, N, K, full):
     # NVFP4_GEMM_PAIR=0 selects the single-CTA persistent kernel where the
