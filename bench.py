@@ -481,7 +481,7 @@ def run_shapes(args, shapes, label):
     hbm_gbs, bf16_tf, src = load_peaks()
     fp4_tf = 4.0 * bf16_tf      # dense FP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
     stream = torch.cuda.Stream()
-    calib = measure_fp4_peak(nv, torch, stream) if label == "saturation" else None
+    calib = measure_fp4_peak(nv, torch, stream) if label in ("saturation", "pages") else None
     rows = []
     for (name, M, Nn, Kk, kind, seed) in shapes:
         us = time_single_shape(nv, torch, dev, M, Nn, Kk, kind, seed, args.steps, stream)
@@ -629,7 +629,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain"], default="attn",
+    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain", "pages"], default="attn",
                     help="attn (default) prints the benchmark line; the others print a per-shape report")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -650,7 +650,7 @@ def main():
             elif args.workload == "chain":
                 print(json.dumps(run_chain(args)), flush=True)
             else:
-                shapes = synth.moe_sweep() if args.workload == "moe" else synth.saturation_sweep()
+                shapes = {"moe": synth.moe_sweep, "pages": synth.pages_sweep}.get(args.workload, synth.saturation_sweep)()
                 print(json.dumps(run_shapes(args, shapes, args.workload)), flush=True)
         return
 

@@ -121,6 +121,18 @@ def saturation_sweep():
     return [(f"sat_{m}x{n}x{k}", m, n, k, "uniform", 1300 + i) for i, (m, n, k) in enumerate(SATURATION_SHAPES)]
 
 
+# The six shapes of the results table in "Peeling the Kernel Onion" (section
+# "The Results": MoE up-projection at 2K/4K/8K batch, attention QKV at
+# 1K/2K/4K batch), for a like-for-like comparison with the numbers printed
+# there for another GPU.
+PAGES_RESULT_SHAPES = [(2048, 2048, 6144), (4096, 2048, 6144), (8192, 2048, 6144),
+                       (1024, 6144, 6144), (2048, 6144, 6144), (4096, 6144, 6144)]
+
+
+def pages_sweep():
+    return [(f"pages_{m}x{n}x{k}", m, n, k, "uniform", 1350 + i) for i, (m, n, k) in enumerate(PAGES_RESULT_SHAPES)]
+
+
 def source(kind: str, M: int, N: int, K: int, seed: int):
     """fp32 (A [M,K], B [N,K]) for a named source kind."""
     if kind == "normal":
