@@ -630,10 +630,13 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     // scratch first.
     const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
     const Plan plan = make_plan(M, N, K, info, sfr);
-    // 256-wide tiles filling at least half the SMs: the CTA-pair kernel
-    // (measured faster than one 128 x 256 tile per CTA from 2048 x 2048 up).
-    if (K % 256 == 0 && !plan.swap && plan.splits == 1 && plan.bq == 256 && M >= 256 &&
-        2 * plan.tiles_p * plan.tiles_q >= info->num_sms && pair_kernel_enabled() && !plan_override().set)
+    // Enough 128 x 256 tiles to fill the SMs twice over: the CTA-pair kernel
+    // on 256 x 256 tiles (measured faster than the split-K and single-CTA
+    // persistent plans from 512 x 6144 and 768 x 4096 up, and on every
+    // saturation shape).
+    if (K % 256 == 0 && !plan.swap && plan.splits == 1 && M >= 512 && N >= 512 &&
+        2 * ((M + 127) / 128) * ((N + 255) / 256) >= info->num_sms && pair_kernel_enabled() &&
+        !plan_override().set)
         return pair_gemm(dev, info, A, sA, B, sB, alpha, D, M, N, K, stream);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;

@@ -377,8 +377,9 @@ def boundary_samples(M, N, seed, n_random=4000, edge=256):
     (2304, 4352, 2048, False),    # 9 x 17 pair tiles, long K
     (1025, 4352, 256, False),     # one K tile per tile; the last tile row holds a single row of A
     (1280, 9000, 768, False),     # last tile column holds 40 columns: the second CTA's B rows all past N
-    (2048, 2048, 6144, False),    # 64 tiles on 74 pairs: every tile cut by K between pairs (stream-K)
-    (1800, 1544, 2048, False),    # stream-K with ragged M and N (8 valid columns in the last tile column)
+    (2048, 2048, 6144, False),    # 64 pair tiles on 74 pairs, long K
+    (1800, 1544, 2048, False),    # ragged M and N (8 valid columns in the last tile column)
+    (520, 6144, 512, False),      # a mid-size M on pair tiles: the last tile row holds 8 rows
 ])
 def test_gemm_persistent_path_matches_oracle(nv, monkeypatch, pair, M, N, K, full):
     # NVFP4_GEMM_PAIR=0 selects the single-CTA persistent kernel where the
