@@ -39,11 +39,14 @@
  *   - Arguments are validated on the host before anything is launched; a
  *     failed check returns a status and launches nothing.  No exception or
  *     abort crosses this boundary.
- *   - The library owns per-device, per-stream scratch (re-laid-out scales,
- *     split-K partial sums) which it allocates on first need and grows; the
- *     first call of a new, larger shape on a stream may therefore call
- *     cudaMalloc, so make it before capturing that stream into a CUDA graph.
- *     Calls on different streams use different scratch and may overlap.
+ *   - The library owns per-device, per-stream scratch (scales re-laid out for
+ *     the tensor cores, when a call needs that) and a 4 KB block of counters
+ *     per stream for the grouped GEMM's run-time work hand-out, which it
+ *     allocates on first need; scratch grows with the shapes.  The first call
+ *     of a new, larger shape on a stream may therefore call cudaMalloc, so
+ *     make it before capturing that stream into a CUDA graph.  Calls on
+ *     different streams use different scratch and counters and may overlap;
+ *     calls on one stream run in stream order.
  *   - Device-side waits are bounded; a wait that runs out records
  *     NVFP4_ERR_TIMEOUT in a device error word read by nvfp4_get_device_error.
  *   - Requires an sm_100 device (B200/GB200); others get
