@@ -585,38 +585,51 @@ def run_chain(args, layers=8):
         torch.cuda.synchronize()
         bufs = [torch.empty((m, dims[li % 2][0]), dtype=torch.bfloat16, device=dev) for li in range(layers)]
 
-        def enqueue():
+        def enqueue(fused):
             a = X
             for li in range(layers):
-                cq, sq = nv.quantize_scaled(a, g_act[li], stream=stream)
                 cb, sb, gb = weights[li]
-                nv.gemm(cq, sq, cb, sb, g_act[li] * gb, out=bufs[li], stream=stream)
+                if fused:   # the GEMM quantizes its activation tiles (one launch per layer where the shape allows)
+                    nv.gemm_bf16a(a, g_act[li], cb, sb, g_act[li] * gb, out=bufs[li], stream=stream)
+                else:
+                    cq, sq = nv.quantize_scaled(a, g_act[li], stream=stream)
+                    nv.gemm(cq, sq, cb, sb, g_act[li] * gb, out=bufs[li], stream=stream)
                 a = bufs[li]
 
-        with torch.cuda.stream(stream):
-            enqueue()
-        stream.synchronize()
-        g_chain = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_chain, stream=stream):
-            enqueue()
-        reps = max(3, min(args.steps, 200))
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                g_chain.replay()
-        stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(reps):
-                g_chain.replay()
-            e1.record(stream)
-        stream.synchronize()
-        assert nv.get_device_error(stream) == 0
-        us_layer = e0.elapsed_time(e1) * 1e3 / (reps * layers)
+        def time_chain(fused):
+            with torch.cuda.stream(stream):
+                enqueue(fused)
+            stream.synchronize()
+            g_chain = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_chain, stream=stream):
+                enqueue(fused)
+            reps = max(3, min(args.steps, 200))
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    g_chain.replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g_chain.replay()
+                e1.record(stream)
+            stream.synchronize()
+            assert nv.get_device_error(stream) == 0
+            return e0.elapsed_time(e1) * 1e3 / (reps * layers)
+
+        us_two = time_chain(False)
+        os.environ["NVFP4_GEMM_FUSE_QUANT"] = "1"
+        try:
+            us_fused = time_chain(True)
+        finally:
+            os.environ.pop("NVFP4_GEMM_FUSE_QUANT", None)
         b = sum(accounting.gemm_bytes(m, dims[li % 2][0], dims[li % 2][1]) for li in range(layers)) / layers
-        out.append({"M": m, "us_per_layer": round(us_layer, 2), "GBps": round(b / us_layer / 1e3, 1)})
-    return {"workload": f"dependent chain of {layers} layers (quantize_scaled + GEMM), shapes alternating "
-                        f"Mx{N}x{K} and Mx{K}x{N}, one CUDA graph, programmatic dependent launch",
+        out.append({"M": m, "us_per_layer": round(us_two, 2), "GBps": round(b / us_two / 1e3, 1),
+                    "us_per_layer_fused": round(us_fused, 2)})
+    return {"workload": f"dependent chain of {layers} layers (quantize_scaled + GEMM; `_fused`: nvfp4_gemm_bf16a "
+                        f"with NVFP4_GEMM_FUSE_QUANT=1, the GEMM quantizing its own activation tiles), "
+                        f"shapes alternating Mx{N}x{K} and Mx{K}x{N}, one CUDA graph, programmatic dependent launch",
             "layers": layers, "per_M": out,
             "note": "weights 6.3 MB per layer stay in L2 across replays (the chain is launch- and "
                     "latency-bound, which is what it measures)"}

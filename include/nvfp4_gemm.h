@@ -205,6 +205,29 @@ nvfp4_status nvfp4_quantize_scaled(const void* X, int x_is_bf16, int rows, int K
                                    void* scales, void* stream);
 
 /*
+ * nvfp4_gemm_bf16a -- the GEMM with BF16 activations, quantized inside the
+ * call with the given global scale gA (the quantize-and-pack of
+ * nvfp4_quantize_scaled, then nvfp4_gemm), so that decode feeds the GEMM
+ * straight from the previous layer's BF16 output ("Peeling the Kernel Onion",
+ * section "The Critical Connection to Real Inference").
+ *   A      BF16 [M][K], row-major, 16-byte aligned.
+ *   gA     the activations' global scale, positive and finite.
+ *   B, sB  the NVFP4 weights as for nvfp4_gemm; alpha = gA * gB as there.
+ *   D      BF16 [M][N].
+ * The activations are quantized into per-stream scratch by the one-launch
+ * quantizer, then the GEMM runs (two launches, chained by programmatic
+ * dependent launch).  With the environment variable NVFP4_GEMM_FUSE_QUANT=1,
+ * for M <= 64 with K a multiple of 256 and 16-byte aligned sB, the GEMM
+ * kernel instead quantizes each activation tile in shared memory (one launch;
+ * slower on the attention shapes, where every CTA of a weight-tile column
+ * repeats the conversion).  Either way the result equals
+ * nvfp4_quantize_scaled followed by nvfp4_gemm on the same stream.  Errors as for nvfp4_gemm, plus
+ * NVFP4_ERR_INVALID_ARG for gA not positive and finite.
+ */
+nvfp4_status nvfp4_gemm_bf16a(const void* A, float gA, const void* B, const void* sB, float alpha, void* D, int M,
+                              int N, int K, void* stream);
+
+/*
  * nvfp4_fp4_peak_probe -- calibration of the dense FP4 tensor-core rate (no
  * counterpart on the pages, which quote only a vendor-style peak for another
  * GPU, "Peeling the Kernel Onion", section "The Results").  Launches one CTA

@@ -32,7 +32,7 @@ EXPORTS = (
     "nvfp4_gemm", "nvfp4_gemm_ex", "nvfp4_grouped_gemm", "nvfp4_quantize", "nvfp4_swizzle_scales",
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
-    "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe", "nvfp4_quantize_scaled",
+    "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe", "nvfp4_quantize_scaled", "nvfp4_gemm_bf16a",
 )
 
 
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_fp4_peak_probe.restype = i32
         L.nvfp4_quantize_scaled.argtypes = [P, i32, i32, i32, f32, P, P, P]
         L.nvfp4_quantize_scaled.restype = i32
+        L.nvfp4_gemm_bf16a.argtypes = [P, f32, P, P, f32, P, i32, i32, i32, P]
+        L.nvfp4_gemm_bf16a.restype = i32
         _lib = L
     return _lib
 
@@ -190,6 +192,27 @@ def grouped_gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.T
     _check(lib().nvfp4_grouped_gemm(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), alpha.data_ptr(),
                                     row_offsets.data_ptr(), G, out.data_ptr(), Mt, N, K, _stream(stream)),
            "nvfp4_grouped_gemm")
+    return out
+
+
+def gemm_bf16a(A: torch.Tensor, gA: float, B: torch.Tensor, sB: torch.Tensor, alpha: float,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """D = the NVFP4 GEMM of BF16 activations A [M, K] (quantized inside the
+    call with global scale gA) and weights B [N, K/2], sB [N, K/16]."""
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A must be [M, K] BF16 and B [N, K/2]")
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] * 2 != K:
+        raise ValueError(f"K mismatch: A holds K={K}, B holds K={B.shape[1] * 2}")
+    _need(A, "A", torch.bfloat16, (M, K))
+    _need(B, "B", torch.uint8, (N, K // 2))
+    _need(sB, "sB", torch.uint8, (N, K // 16))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _need(out, "out", torch.bfloat16, (M, N))
+    _check(lib().nvfp4_gemm_bf16a(A.data_ptr(), float(gA), B.data_ptr(), sB.data_ptr(), float(alpha), out.data_ptr(),
+                                  M, N, K, _stream(stream)), "nvfp4_gemm_bf16a")
     return out
 
 

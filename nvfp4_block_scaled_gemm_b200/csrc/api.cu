@@ -76,10 +76,11 @@ struct Scratch {
     size_t cap = 0;
 };
 std::map<std::pair<int, uintptr_t>, Scratch> g_scratch;
+std::map<std::pair<int, uintptr_t>, Scratch> g_act_scratch;   // quantized activations (nvfp4_gemm_bf16a)
 
-nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** out) {
+nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** out, bool act = false) {
     std::lock_guard<std::mutex> lk(g_mu);
-    Scratch& s = g_scratch[{dev, reinterpret_cast<uintptr_t>(stream)}];
+    Scratch& s = (act ? g_act_scratch : g_scratch)[{dev, reinterpret_cast<uintptr_t>(stream)}];
     if (s.cap < bytes) {
         size_t want = std::max(bytes, s.cap * 2);
         want = (want + 0xFFFFF) & ~size_t(0xFFFFF);
@@ -173,6 +174,20 @@ bool make_scale_map(CUtensorMap* map, const void* base, long long rows, long lon
     const cuuint32_t box[2] = {16u, (cuuint32_t)box_rows};
     const cuuint32_t elem_strides[2] = {1u, 1u};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over row-major BF16 [rows][cols]; box 256 values (one 256-element
+// K tile, 512 bytes) x box_rows, no swizzle (the writer warps read it).
+bool make_bf16_map(CUtensorMap* map, const void* base, long long rows, long long cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {256u, (cuuint32_t)box_rows};
+    const cuuint32_t elem_strides[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -325,11 +340,11 @@ struct Maps {
     CUtensorMap p, q, sp, sq;
 };
 
-template <int BQ, bool SWAP, bool SPLITK, bool SFR>
+template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false>
 nvfp4_status launch_gemm_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, const GemmParams& prm, dim3 grid,
                                 cudaStream_t stream) {
-    using C = TileConfig<BQ, SPLITK>;
-    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK, SFR>;
+    using C = TileConfig<BQ, SPLITK, QBF16>;
+    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK, SFR, QBF16>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!(info->smem_attr_set & bit)) {
@@ -822,6 +837,64 @@ nvfp4_status nvfp4_quantize_scaled(const void* X, int x_is_bf16, int rows, int K
         return NVFP4_ERR_CUDA;
     }
     return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gemm_bf16a(const void* A, float gA, const void* B, const void* sB, float alpha, void* D, int M,
+                              int N, int K, void* stream_) {
+    if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!(gA > 0.0f) || !std::isfinite(gA)) return NVFP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!A || !B || !sB || !D || !aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sB, 4))
+        return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const bool sfr = (K % 256 == 0) && aligned(sB, 16);
+    const Plan plan = make_plan(M, N, K, info, sfr);
+    // The GEMM can quantize its activation tiles itself, but every CTA of a
+    // weight-tile column then repeats the same conversion (IEEE divisions on
+    // the critical path): measured 13.8 against 7.4 us per 768x6144 layer at
+    // M = 1 in a dependent chain.  So the separate one-launch quantizer,
+    // spread over all SMs and overlapped by programmatic dependent launch, is
+    // the default; NVFP4_GEMM_FUSE_QUANT=1 selects the in-kernel form.
+    const char* fuse_env = std::getenv("NVFP4_GEMM_FUSE_QUANT");
+    const bool fuse = fuse_env && fuse_env[0] == '1';
+    if (fuse && sfr && plan.swap && (plan.bq == 16 || plan.bq == 32)) {
+        // Fused: the GEMM quantizes its activation tiles in shared memory.
+        Maps maps;
+        if (!make_operand_map(&maps.p, B, N, K / 2, 128) || !make_bf16_map(&maps.q, A, M, K, plan.bq) ||
+            !make_scale_map(&maps.sp, sB, N, K / 16, 128))
+            return NVFP4_ERR_CUDA;
+        maps.sq = maps.sp;   // unused: the Q scales are computed in the kernel
+        GemmParams prm{};
+        prm.D = static_cast<__nv_bfloat16*>(D);
+        prm.alpha = alpha;
+        prm.rows_p = N;
+        prm.rows_q = M;
+        prm.K = K;
+        prm.ldd = N;
+        prm.k_tiles = plan.k_tiles;
+        prm.tiles_q = plan.tiles_q;
+        prm.gq = gA;
+        const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
+        const int sk = plan.splits > 1 ? 1 : 0;
+        if (plan.bq == 16)
+            return sk ? launch_gemm_kernel<16, true, true, true, true>(info, 1ull << 40, maps, prm, grid, stream)
+                      : launch_gemm_kernel<16, true, false, true, true>(info, 1ull << 41, maps, prm, grid, stream);
+        return sk ? launch_gemm_kernel<32, true, true, true, true>(info, 1ull << 42, maps, prm, grid, stream)
+                  : launch_gemm_kernel<32, true, false, true, true>(info, 1ull << 43, maps, prm, grid, stream);
+    }
+    // Quantize into per-stream scratch, then the GEMM (two launches, chained
+    // by programmatic dependent launch).
+    const size_t codes_bytes = (size_t)M * (K / 2), off_s = align_up(codes_bytes, 256);
+    uint8_t* ws = nullptr;
+    if ((st = get_scratch(dev, stream, off_s + (size_t)M * (K / 16), &ws, /*act=*/true)) != NVFP4_OK) return st;
+    if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if ((st = nvfp4_quantize_scaled(A, 1, M, K, gA, ws, ws + off_s, stream_)) != NVFP4_OK) return st;
+    return nvfp4_gemm(ws, ws + off_s, B, sB, alpha, D, M, N, K, stream_);
 }
 
 nvfp4_status nvfp4_fp4_peak_probe(int pair, long long steps, int* ctas_out, void* stream_) {

@@ -52,6 +52,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace nvfp4 {
 
@@ -64,7 +65,10 @@ constexpr int kThreads = 192;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 constexpr int kScaleBuffers = 4;    // rotating TMEM scale buffers
 
-template <int BQ, bool SPLITK>
+// QBF16: the Q operand (the activations, swapped layout) arrives as BF16 and
+// is quantized in shared memory by the writer warps: each stage also holds
+// the raw BF16 tile, BQ rows x 256 values.
+template <int BQ, bool SPLITK, bool QBF16 = false>
 struct TileConfig {
     static_assert(BQ == 16 || BQ == 32 || BQ == 64 || BQ == 128 || BQ == 256, "BQ");
     static constexpr int P_BYTES = kBM * kStageKBytes;
@@ -72,7 +76,9 @@ struct TileConfig {
     static constexpr int Q_BLOCKS = BQ > 128 ? BQ / 128 : 1;        // 128-row scale blocks of Q
     static constexpr int SFP_BYTES = 4 * kAtomBytes;
     static constexpr int SFQ_BYTES = 4 * kAtomBytes * Q_BLOCKS;
-    static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
+    static constexpr int QRAW_OFF = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
+    static constexpr int QRAW_BYTES = QBF16 ? BQ * 256 * 2 : 0;
+    static constexpr int STAGE_BYTES = QRAW_OFF + QRAW_BYTES;
     // split-K receive slots: one fp32 row of kPartLd floats per tile row, in
     // a region of their own when that still leaves kScaleBuffers stages,
     // otherwise in the ring (then written only after the whole cluster's
@@ -106,6 +112,7 @@ struct GemmParams {
     int k_tiles;              // ceil(K / 256)
     int tiles_q;              // tiles along Q; blockIdx.y = tq + tiles_q * tp
     int prefetch_b;           // B is constant: fetch its first tiles before waiting on the previous grid
+    float gq;                 // QBF16: global scale of the BF16 activations
 };
 
 template <int BQ, bool SWAP>
@@ -221,20 +228,22 @@ __device__ __forceinline__ void reduce_owned_rows(const GemmParams& prm, uint32_
     }
 }
 
-template <int BQ, bool SWAP, bool SPLITK, bool SFR>
+template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                       const GemmParams prm) {
-    using C = TileConfig<BQ, SPLITK>;
+    static_assert(!QBF16 || (SWAP && SFR && BQ <= 64), "BF16 activations: swapped layout, row-major scale tiles");
+    using C = TileConfig<BQ, SPLITK, QBF16>;
     constexpr int S = C::STAGES;
     constexpr int NB = kScaleBuffers;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // [ring: S stages][split-K receive slots][barriers]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES + C::SLOT_BYTES);
-    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB] accum
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + NB + 1);
+    // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB] accum,
+    //       [2S+NB+1] cvt (QBF16: the four writer warps quantized a K tile)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + NB + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -250,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };
     auto sf_ready_bar = [&](int b) { return bar_base + 8u * (2 * S + b); };
     const uint32_t accum_bar = bar_base + 8u * (2 * S + NB);
+    const uint32_t cvt_bar = bar_base + 8u * (2 * S + NB + 1);
 
     // Q scale blocks that exist in the (row-padded) atom buffer for this tile.
     const int q_row0 = tq * BQ;
@@ -265,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < NB; ++b) mbar_init(sf_ready_bar(b), 4);
         mbar_init(accum_bar, 1);
+        mbar_init(cvt_bar, 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -303,13 +314,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_q = policy_evict_last();
             // With a constant B, its first ring's worth of tiles is requested
             // before waiting for the previous grid (only B is touched then).
+            // bytes of one stage: P tile + P scales + the Q side (FP4 tile and
+            // scales, or the raw BF16 tile that the writers quantize)
+            constexpr uint32_t kStageTx =
+                C::P_BYTES + 16 * kBM + (QBF16 ? (uint32_t)C::QRAW_BYTES : (uint32_t)(C::Q_BYTES + 16 * BQ));
+            auto load_q = [&](uint32_t st, uint32_t bar, int kt) {
+                if (QBF16) {
+                    tma_load_2d(st + C::QRAW_OFF, &tmQ, bar, kt * 256, q_row0, pol_q);
+                } else {
+                    tma_load_2d(st + C::P_BYTES, &tmQ, bar, kt * kStageKBytes, q_row0, pol_q);
+                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, bar, kt * 16, q_row0, pol_q);
+                }
+            };
             int pre = 0;
             if (SFR && prm.prefetch_b) {
                 pre = min(S, kt_end - kt_begin);
                 for (int i = 0; i < pre; ++i) {
                     const int kt = kt_begin + i;
                     const uint32_t st = smem_base + i * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(full_bar(i), C::P_BYTES + C::Q_BYTES + 16 * kBM + 16 * BQ);
+                    mbar_arrive_expect_tx(full_bar(i), kStageTx);
                     if (SWAP) {   // B is P
                         tma_load_2d(st, &tmP, full_bar(i), kt * kStageKBytes, tp * kBM, pol_p);
                         tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(i), kt * 16, tp * kBM, pol_p);
@@ -328,9 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t st = smem_base + s * C::STAGE_BYTES;
                 if (it < pre) {   // the other operand of a prefetched stage
                     if (SWAP) {
-                        tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
-                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(s), kt * 16, q_row0,
-                                    pol_q);
+                        load_q(st, full_bar(s), kt);
                     } else {
                         tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
                         tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
@@ -340,12 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) break;
                 if (SFR) {
                     // row-major scale tiles: 16 bytes (= 4 K steps) per row
-                    mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + C::Q_BYTES + 16 * kBM + 16 * BQ);
+                    mbar_arrive_expect_tx(full_bar(s), kStageTx);
                     tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
-                    tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
                     tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
-                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(s), kt * 16, q_row0,
-                                pol_q);
+                    load_q(st, full_bar(s), kt);
                 } else {
                     const int steps = min(4, steps_total - 4 * kt);
                     const uint32_t sf_bytes = (uint32_t)steps * kAtomBytes;
@@ -408,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (j0 < 0 || mbar_wait(empty_bar(j0 % S), (uint32_t)(j0 / S) & 1u, abort_flag));
                     // take the following K tiles that have landed too, up to half
                     // the scale buffers, so the MMA keeps the other half busy
-                    while (got && cnt < NB / 2 && kt + cnt < kt_end) {
+                    while (got && !QBF16 && cnt < NB / 2 && kt + cnt < kt_end) {
                         const int i1 = it + cnt, s1 = i1 % S, j1 = i1 - NB;
                         if (!mbar_test(full_bar(s1), (uint32_t)(i1 / S) & 1u) ||
                             (j1 >= 0 && !mbar_test(empty_bar(j1 % S), (uint32_t)(j1 / S) & 1u)))
@@ -418,6 +437,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
                 cnt = __shfl_sync(0xffffffffu, cnt, 0);
+                if (QBF16) {
+                    // Quantize this K tile's BF16 activations (BQ rows x 16
+                    // blocks of 16) into the FP4 Q tile, in the 128-byte
+                    // swizzled K-major layout the MMA descriptor reads, and
+                    // their scales into the row-major scale tile; then make
+                    // the writes visible to the tensor cores and wait for the
+                    // other writer warps' rows.
+                    const uint32_t st = smem_base + (it % S) * C::STAGE_BYTES;
+                    const uint32_t raw = st + C::QRAW_OFF, qt = st + C::P_BYTES;
+                    const uint32_t sq = st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES;
+                    const float gq = prm.gq, six_gq = __fmul_rn(6.0f, prm.gq);
+                    for (int bidx = (warp - 2) * 32 + lane; bidx < BQ * 16; bidx += 128) {
+                        const int r = bidx >> 4, kb = bidx & 15;
+                        float x[16];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint4 v = ld_shared_v4(raw + (uint32_t)(r * 512 + kb * 32 + 16 * h));
+                            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                x[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
+                                x[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+                            }
+                        }
+                        uint32_t sc, cd[2];
+                        quantize_block16(x, gq, six_gq, sc, cd);
+                        const uint32_t dst = qt + (uint32_t)(r * 128 + ((((kb >> 1) ^ (r & 7)) << 4) | ((kb & 1) << 3)));
+                        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(dst), "r"(cd[0]), "r"(cd[1]) : "memory");
+                        asm volatile("st.shared.u8 [%0], %1;" ::"r"(sq + (uint32_t)(r * 16 + kb)), "h"((uint16_t)sc)
+                                     : "memory");
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    int cv = 1;
+                    if (lane == 0) {
+                        mbar_arrive(cvt_bar);
+                        cv = mbar_wait(cvt_bar, (uint32_t)it & 1u, abort_flag) ? 1 : 0;
+                    }
+                    if (!__shfl_sync(0xffffffffu, cv, 0)) break;
+                }
                 for (int u = 0; u < cnt; ++u) {
                     const int iu = it + u;
                     const uint32_t st = smem_base + (iu % S) * C::STAGE_BYTES;

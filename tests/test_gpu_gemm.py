@@ -92,6 +92,37 @@ def test_quantize_scaled_then_gemm_chain(nv):
         assert not violations(D.float().cpu().numpy(), ref, ad).any()
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (1, 768, 6144), (8, 768, 6144), (16, 2048, 1024),   # one 16-row activation tile (fused)
+    (33, 768, 2048), (64, 256, 6144),                   # 32-row tiles, two of them at M=64 (fused)
+    (100, 520, 1024),                                    # beyond the swapped plans: quantize, then GEMM
+    (7, 264, 320)])                                      # K % 256 != 0: quantize, then GEMM
+@pytest.mark.parametrize("fuse", ["0", "1"])
+def test_gemm_bf16a_matches_quantize_then_gemm(nv, monkeypatch, fuse, M, N, K):
+    # BF16 activations quantized inside nvfp4_gemm_bf16a (by the separate
+    # quantizer, or with NVFP4_GEMM_FUSE_QUANT=1 by the GEMM kernel where the
+    # shape allows) give the same bits as nvfp4_quantize_scaled followed by
+    # nvfp4_gemm, and the oracle's result within the bound.
+    monkeypatch.setenv("NVFP4_GEMM_FUSE_QUANT", fuse)
+    X = synth.activations_with_outliers(M, K, 500 + M)
+    A = dev(X).to(torch.bfloat16)
+    Xb = A.float().cpu().numpy()
+    ga = float(np.float32(oracle.quantize(Xb)[2]))
+    W = synth.normal(N, K, 600 + N, std=0.02)
+    cb, sb, gb = oracle.quantize(W)
+    B, SB = dev(cb), dev(sb)
+    alpha = float(np.float32(ga) * np.float32(gb))
+    ca, sa = oracle.quantize_with_scale(Xb, ga)
+    _, ref, ad = oracle.gemm(ca, sa, cb, sb, alpha, M, N, K)
+    D1 = nv.gemm_bf16a(A, ga, B, SB, alpha)
+    qa, qs = nv.quantize_scaled(A, ga)
+    D2 = nv.gemm(qa, qs, B, SB, alpha)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    assert torch.equal(D1.view(torch.int16), D2.view(torch.int16))
+    assert not violations(D1.float().cpu().numpy(), ref, ad).any()
+
+
 def test_quantize_scaled_rejects_bad_arguments(nv):
     X = torch.ones((4, 32), device="cuda")
     for g in (0.0, -1.0, float("inf"), float("nan")):
