@@ -43,10 +43,18 @@
 // peer has started is arrived at kernel start and waited on just before the
 // first remote store.
 //
+// BF16 activations (QBF16, swapped layout only): the producer brings the raw
+// BF16 Q tile (BQ rows x 256 values) by TMA instead of the FP4 tile and its
+// scales; the four writer warps quantize it (quant.cuh block steps) into the
+// 128-byte swizzled FP4 tile and the row-major scale tile of the stage, fence
+// the writes for the tensor cores, meet on the cvt barrier, and then move the
+// scales into TMEM as usual.
+//
 // Barriers: full[s] (producer arrive + TMA bytes), empty[s] (MMA commit:
 // stage s may be refilled and the TMEM scale buffer of that K tile may be
 // rewritten), sf_ready[b] (4 writer arrivals: scale buffer b holds this K
-// tile), accum (MMA commit after the last K tile).  Every wait is bounded.
+// tile), accum (MMA commit after the last K tile), cvt (QBF16: 4 writer
+// arrivals per K tile).  Every wait is bounded.
 #pragma once
 
 #include <cuda_bf16.h>

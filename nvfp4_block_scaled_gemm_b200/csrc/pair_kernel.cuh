@@ -48,8 +48,9 @@
 // MMA issuer (CTA 0), warps 2..5 epilogue, warps 6..9 scale writers, warp 10
 // scale producer.  Warps w and w + 4 share TMEM lane quadrant w % 4.
 //
-// Used for the compute-bound shapes of "Peeling the Kernel Onion" (section
-// "The Benchmark Design"); K a multiple of 256.
+// Used for the compute-bound shapes of "Peeling the Kernel Onion" (sections
+// "The Benchmark Design" and "The Results"), from M, N >= 512 with enough
+// 128 x 256 tiles for two per SM; K a multiple of 256.
 #pragma once
 
 #include "persistent_kernel.cuh"

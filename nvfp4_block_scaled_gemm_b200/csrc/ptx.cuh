@@ -255,13 +255,6 @@ __device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc
         : "memory");
 }
 
-// Copy a 32-row x 16-byte block of shared memory (described by `sdesc`) to
-// TMEM lanes 0..31, columns taddr..taddr+3, replicated into all four lane
-// quadrants.
-__device__ __forceinline__ void tc_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 // D(tmem) (+)= (A * sfA) x (B * sfB)^T for one K=64 step of E2M1 operands with
 // UE4M3 scales, one scale per 16 elements.
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -332,16 +325,6 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
     return d;
 }
 
-// A 512-byte scale atom: 32 rows of 16 bytes, unswizzled, i.e. four 8-row x
-// 16-byte core matrices 128 bytes apart (both offset fields 128 B).
-__device__ __forceinline__ uint64_t desc_scale_atom(uint32_t saddr) {
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)(128 >> 4) << 16;
-    d |= (uint64_t)(128 >> 4) << 32;
-    d |= (uint64_t)1 << 46;
-    return d;
-}
-
 // Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format code 1),
 // both K-major, UE4M3 scales (bit 23 = 0), dense K = 64, M in bits 24-28
 // (M >> 4), N in bits 17-22 (N >> 3).
@@ -362,10 +345,6 @@ __device__ __forceinline__ void grid_launch_dependents() {
 }
 
 // --------------------------------------------------------------- misc
-__device__ __forceinline__ void named_barrier(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
