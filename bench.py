@@ -288,8 +288,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         sweep.append({"M": m, "us": round(us, 3), "GBps": round(b / us / 1e3, 1), "TFLOPS": round(f / us / 1e6, 2),
                       "hbm_frac": round(b / us / 1e3 / hbm_gbs, 4)})
 
-    # Roofline of the dominant kernel (the GEMM kernel: every launch in a step
-    # is one GEMM launch).  Average launch duration over the timed region.
+    # Roofline of the step's GEMM launches (one launch per GEMM: the CUDA-core
+    # kernel for M = 1, the tensor-core kernel for the other five, which
+    # dominates the time).  Average launch duration over the timed region.
     launches_per_rank = launches
     avg_launch_us = ms * 1e3 / max(1, launches_per_rank)
     bytes_per_launch = step_bytes() / len(SWEEP_M)
@@ -313,6 +314,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(achieved / hbm_gbs, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} hbm_gbs",
+                     "kernel": "nvfp4_gemm_kernel (M = 16..512) and nvfp4_gemv_kernel (M = 1), one launch per GEMM",
                      "per_launch": {"algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_launch_us, 3)}},
         "e2e": e2e,
         "gpu_launches": launches_per_rank,

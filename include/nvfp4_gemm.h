@@ -80,8 +80,16 @@ typedef enum {
  *   D [M][N] bf16: device, written.
  *   Requirements: M >= 0, N >= 0, K > 0; K % 64 == 0; N % 8 == 0; A, B, D
  *   16-byte aligned; sA, sB 4-byte aligned.  M == 0 or N == 0 is a no-op.
- * Small M uses the weight-streaming kernel (B rows on the tensor cores' M
- * side, split-K over the SMs); large M uses 128 x N-tile output tiles.
+ * One or two token rows (up to four for small N, K >= 4096 beyond one) run
+ * on the CUDA cores: a matrix-vector kernel that streams B straight into
+ * registers, whose block sums are exact and whose fp32 sum over the K/16
+ * blocks is the only rounding before alpha and the BF16 store.  Other small
+ * M uses the weight-streaming tensor-core kernel (B rows on the MMA's M side,
+ * split-K over a thread-block cluster); large M uses 128- or 256-row output
+ * tiles, on CTA pairs for the largest shapes.  Environment switches, for
+ * tuning and tests: NVFP4_GEMM_GEMV=0 keeps every M on the tensor cores and
+ * NVFP4_GEMM_GEMV=<n> sends every M <= n (at most 16) to the CUDA cores;
+ * NVFP4_GEMM_PAIR=0 keeps large shapes off the CTA-pair kernel.
  */
 nvfp4_status nvfp4_gemm(const void* A, const void* sA,
                         const void* B, const void* sB,

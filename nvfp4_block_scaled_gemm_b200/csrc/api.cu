@@ -17,6 +17,7 @@
 #include "../../include/nvfp4_gemm.h"
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
+#include "gemv_kernel.cuh"
 #include "grouped_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "peak_kernel.cuh"
@@ -441,6 +442,100 @@ bool pair_kernel_enabled() {
     return !(e && e[0] == '0');
 }
 
+// Whether nvfp4_gemm runs the CUDA-core kernel for a few activation rows
+// (nvfp4_gemv_kernel) instead of the tensor-core kernels.  Measured on
+// graph-replayed back-to-back calls (us per call, tensor cores -> CUDA cores):
+// M = 1 wins everywhere (768x6144 5.8 -> 2.7, 2048x6144 7.2 -> 3.6,
+// 8192x8192 12.9 -> 11.3, 6144x768 5.5 -> 4.3); M = 2 wins with K >= 4096 up
+// to N = 2048 (7.2 -> 4.9) and loses at 8192x8192 and at K = 768, where most
+// of a CTA's threads have no K chunk; M = 4 wins only up to N ~ 768 (5.9 ->
+// 4.3); M >= 8 loses.  NVFP4_GEMM_GEMV=0 turns the kernel off;
+// NVFP4_GEMM_GEMV=<n> (1..16) sends every M <= n to it (tuning and tests);
+// NVFP4_GEMM_GEMV_RW=1|2|4 forces the weight rows per CTA.
+bool use_gemv(int M, int N, int K) {
+    if (plan_override().set) return false;
+    if (const char* e = std::getenv("NVFP4_GEMM_GEMV")) {
+        const int v = std::atoi(e);
+        return M <= (v < 0 ? 0 : v > 16 ? 16 : v);
+    }
+    if (M == 1) return true;
+    if (K < 4096) return false;
+    return (M == 2 && N <= 4096) || (M <= 4 && N <= 1024);
+}
+
+// At most as many CTAs as fit on the GPU at once (the kernel walks the rest
+// of the row groups itself).
+template <int MT, int RW>
+nvfp4_status launch_gemv_kernel(DeviceInfo* info, const nvfp4::GemvParams& prm, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemv_kernel<MT, RW>;
+    static const int per_sm = [kern] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, nvfp4::kGemvThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            b = 0;
+        }
+        return b > 0 ? b : 1;
+    }();
+    const int groups = (prm.N + RW - 1) / RW;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(groups, per_sm * info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+template <int MT>
+nvfp4_status launch_gemv_rw(DeviceInfo* info, int rw, const nvfp4::GemvParams& prm, cudaStream_t stream) {
+    switch (rw) {
+        case 1: return launch_gemv_kernel<MT, 1>(info, prm, stream);
+        case 2: return launch_gemv_kernel<MT, 2>(info, prm, stream);
+        default:
+            if constexpr (MT >= 16) return launch_gemv_kernel<MT, 2>(info, prm, stream);   // 4 x 16 would spill
+            else return launch_gemv_kernel<MT, 4>(info, prm, stream);
+    }
+}
+
+// The CUDA-core path for M <= 16.  Weight rows per CTA (measured): one row
+// for a single token row and a small matrix (spread over the most CTAs),
+// four from N = 2048 up, two with two or more token rows (each decoded
+// activation chunk serves both rows).
+nvfp4_status gemv_gemm(DeviceInfo* info, const void* A, const void* sA, const void* B, const void* sB, float alpha,
+                       void* D, int M, int N, int K, unsigned flags, cudaStream_t stream) {
+    nvfp4::GemvParams prm{};
+    prm.A = static_cast<const uint8_t*>(A);
+    prm.sA = static_cast<const uint8_t*>(sA);
+    prm.B = static_cast<const uint8_t*>(B);
+    prm.sB = static_cast<const uint8_t*>(sB);
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.alpha = alpha;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+    int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
+    if (const char* e = std::getenv("NVFP4_GEMM_GEMV_RW")) {
+        const int v = std::atoi(e);
+        if (v == 1 || v == 2 || v == 4) rw = v;
+    }
+    if (M <= 1) return launch_gemv_rw<1>(info, rw, prm, stream);
+    if (M <= 2) return launch_gemv_rw<2>(info, rw, prm, stream);
+    if (M <= 4) return launch_gemv_rw<4>(info, rw, prm, stream);
+    if (M <= 8) return launch_gemv_rw<8>(info, rw, prm, stream);
+    return launch_gemv_rw<16>(info, rw, prm, stream);
+}
+
 nvfp4_status launch_pair(DeviceInfo* info, const CUtensorMap& tmA, const CUtensorMap& tmB,
                          const nvfp4::PairParams& prm, cudaStream_t stream) {
     using C = nvfp4::PairConfig;
@@ -638,6 +733,7 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     st = current_device(&dev, &info);
     if (st != NVFP4_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (use_gemv(M, N, K)) return gemv_gemm(info, A, sA, B, sB, alpha, D, M, N, K, flags, stream);
 
     // Scales go to the kernel row-major (TMA tiles, laid out for the tensor
     // cores inside the kernel) when a 256-element K tile of scales is a
@@ -859,9 +955,11 @@ nvfp4_status nvfp4_gemm_bf16a(const void* A, float gA, const void* B, const void
     // the critical path): measured 13.8 against 7.4 us per 768x6144 layer at
     // M = 1 in a dependent chain.  So the separate one-launch quantizer,
     // spread over all SMs and overlapped by programmatic dependent launch, is
-    // the default; NVFP4_GEMM_FUSE_QUANT=1 selects the in-kernel form.
+    // the default; NVFP4_GEMM_FUSE_QUANT=1 selects the in-kernel form, for
+    // the tensor-core shapes (token rows that the CUDA-core kernel takes are
+    // always quantized first).
     const char* fuse_env = std::getenv("NVFP4_GEMM_FUSE_QUANT");
-    const bool fuse = fuse_env && fuse_env[0] == '1';
+    const bool fuse = fuse_env && fuse_env[0] == '1' && !use_gemv(M, N, K);
     if (fuse && sfr && plan.swap && (plan.bq == 16 || plan.bq == 32)) {
         // Fused: the GEMM quantizes its activation tiles in shared memory.
         Maps maps;
@@ -986,6 +1084,12 @@ nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA, const void* B, co
                                 int M, int N, int K, void* stream_) {
     nvfp4_status st = check_gemm_args(A, sA, B, sB, D, M, N, K);
     if (st != NVFP4_OK || M == 0 || N == 0) return st;
+    if (use_gemv(M, N, K)) {   // no scratch at all
+        int dev;
+        DeviceInfo* info;
+        if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+        return gemv_gemm(info, A, sA, B, sB, alpha, D, M, N, K, 0u, static_cast<cudaStream_t>(stream_));
+    }
     // Scales of both operands, re-laid out, must fit the static scratch.
     const size_t sfa_bytes = nvfp4_swizzled_scale_bytes(M, K);
     const size_t sfb_bytes = nvfp4_swizzled_scale_bytes(N, K);

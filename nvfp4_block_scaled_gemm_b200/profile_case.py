@@ -48,7 +48,7 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
         lines = [ln for ln in f if ln.startswith('"')]
     launches = {}
     for row in csv.DictReader(lines):
-        if "nvfp4_gemm_kernel" not in row["Kernel Name"]:
+        if not any(k in row["Kernel Name"] for k in ("nvfp4_gemm_kernel", "nvfp4_gemv_kernel")):
             continue
         rec = launches.setdefault(int(row["ID"]), {})
         unit = row["Metric Unit"].strip().lower()
@@ -68,7 +68,7 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
         per_us[f"M{m}"] = round(rec["gpu__time_duration.sum"], 2)
     mean = sum(per_read[k] + per_write[k] for k in per_read) / len(per_read)
     out = {
-        "kernel": "nvfp4_gemm_kernel",
+        "kernel": "nvfp4_gemv_kernel (M = 1), nvfp4_gemm_kernel (the other five)",
         "workload": "attention sweep M in {1,16,64,128,256,512}, N=768, K=6144",
         "dram_bytes_per_launch": int(round(mean)),
         "per_shape_dram_read": per_read,
@@ -76,7 +76,7 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
         "per_shape_us_under_ncu": per_us,
         "source_hash": source_hash(),
         "command": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum "
-                   "--clock-control none -k regex:nvfp4_gemm_kernel --csv --log-file traffic_attn.csv "
+                   "--clock-control none -k regex:nvfp4_gem[mv]_kernel --csv --log-file traffic_attn.csv "
                    "python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes attn --iters 2",
     }
     with open(out_path, "w") as f:
