@@ -637,6 +637,49 @@ def run_chain(args, layers=8):
                     "latency-bound, which is what it measures)"}
 
 
+def run_decode(args):
+    """Few token rows: the same shapes through the tensor-core kernel
+    (NVFP4_GEMM_GEMV=0) and through the CUDA-core kernel at each weight-row
+    count per CTA (NVFP4_GEMM_GEMV=16, NVFP4_GEMM_GEMV_RW=1|2|4), plus the
+    default dispatch, each as graph-replayed back-to-back calls over rotating
+    buffers; microseconds per GEMM."""
+    import torch
+    import nvfp4_block_scaled_gemm_b200 as nv
+    dev = torch.device("cuda", 0)
+    nv.lib()
+    hbm_gbs = load_peaks()[0]
+    stream = torch.cuda.Stream()
+    settings = (("tensor_cores", {"NVFP4_GEMM_GEMV": "0"}),
+                ("cuda_cores_rw1", {"NVFP4_GEMM_GEMV": "16", "NVFP4_GEMM_GEMV_RW": "1"}),
+                ("cuda_cores_rw2", {"NVFP4_GEMM_GEMV": "16", "NVFP4_GEMM_GEMV_RW": "2"}),
+                ("cuda_cores_rw4", {"NVFP4_GEMM_GEMV": "16", "NVFP4_GEMM_GEMV_RW": "4"}),
+                ("default", {}))
+    keys = ("NVFP4_GEMM_GEMV", "NVFP4_GEMM_GEMV_RW")
+    saved = {k: os.environ.get(k) for k in keys}
+    rows = []
+    try:
+        for (Nn, Kk) in ((768, 6144), (2048, 6144), (256, 6144), (8192, 8192), (6144, 768)):
+            for M in (1, 2, 4, 8):
+                row = {"M": M, "N": Nn, "K": Kk}
+                for name, env in settings:
+                    for k in keys:
+                        os.environ.pop(k, None)
+                    os.environ.update(env)
+                    us = time_single_shape(nv, torch, dev, M, Nn, Kk, "moe", 1700 + M, min(args.steps, 2000), stream)
+                    row[name] = round(us, 2)
+                row["default_hbm_frac"] = round(accounting.gemm_bytes(M, Nn, Kk) / row["default"] / 1e3 / hbm_gbs, 4)
+                rows.append(row)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    return {"workload": "decode: M in {1,2,4,8} on the attention, MoE and two larger weight shapes, tensor-core vs "
+                        "CUDA-core kernel (us per GEMM, graph-replayed back-to-back calls, rotating buffers > L2)",
+            "hbm_gbs": hbm_gbs, "shapes": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -644,7 +687,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain", "pages"], default="attn",
+    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain", "pages", "decode"],
+                    default="attn",
                     help="attn (default) prints the benchmark line; the others print a per-shape report")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -664,6 +708,8 @@ def main():
                 print(json.dumps(run_grouped(args)), flush=True)
             elif args.workload == "chain":
                 print(json.dumps(run_chain(args)), flush=True)
+            elif args.workload == "decode":
+                print(json.dumps(run_decode(args)), flush=True)
             else:
                 shapes = {"moe": synth.moe_sweep, "pages": synth.pages_sweep}.get(args.workload, synth.saturation_sweep)()
                 print(json.dumps(run_shapes(args, shapes, args.workload)), flush=True)
