@@ -22,15 +22,31 @@ def _sources():
     return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh"))] + [HEADER]
 
 
-def source_hash() -> str:
-    """Short hash of the kernel sources (every file under csrc/): committed
-    profile summaries record it, so a reader can tell whether the counters
-    were taken on the code that is built now."""
+def code_text(src: bytes) -> bytes:
+    """Source text with comments removed and whitespace runs collapsed, so
+    that an edit to comments alone does not change the hash."""
+    import re
+    text = src.decode("utf-8", "replace")
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", " ", text).strip().encode()
+
+
+def source_hash(read=None) -> str:
+    """Short hash of the kernel code (every file under csrc/, comments and
+    layout ignored): committed profile summaries record it, so a reader can
+    tell whether the counters were taken on the code that is built now.
+    `read(name)` may supply a file's bytes (for a tree other than the
+    working copy)."""
     import hashlib
     h = hashlib.sha256()
     for f in sorted(os.listdir(CSRC)):
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        if read is None:
+            with open(os.path.join(CSRC, f), "rb") as fh:
+                data = fh.read()
+        else:
+            data = read(f)
+        h.update(f.encode() + code_text(data))
     return h.hexdigest()[:16]
 
 

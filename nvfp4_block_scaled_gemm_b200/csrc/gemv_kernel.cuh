@@ -1,10 +1,13 @@
 // NVFP4 GEMM for a handful of activation rows (decode, M <= 16) on the CUDA
 // cores.
 //
-// With one to a few token rows the GEMM is a matrix-vector product bound by
-// the weight bytes ("Peeling the Kernel Onion", section "The Chain of
-// Reasoning": batch-1 decode reads every weight once for two FLOPs per
-// element), and a 3 MB weight matrix is half a microsecond of HBM time.  The
+// With one to a few token rows the GEMM is a matrix-vector product: two
+// FLOPs per weight element read, so it is bound by the weight bytes (small-
+// batch decode is memory-bound: "The SM120 FP4 Kernel Disaster", section
+// "Finding 4: Memory Bandwidth Is the Real Wall"; the batch-1 attention and
+// MoE projections are the first shapes measured in "Peeling the Kernel
+// Onion", section "The Chain of Reasoning"), and a 3 MB weight matrix is half
+// a microsecond of HBM time.  The
 // tensor-core kernels spend several microseconds per call in hand-offs
 // (tensor map fetch, TMA, TMEM scale stores, MMA, split-K exchange through
 // distributed shared memory); this kernel has none of them: every thread
