@@ -67,6 +67,14 @@ def lib():
         L.oracle_swizzle_scales.argtypes = [P, i32, i32, P]
         L.oracle_dot.restype = ctypes.c_uint16
         L.oracle_dot.argtypes = [P, P, P, P, i32, f32, P, P]
+        L.oracle_sparse24_compress.restype = i32
+        L.oracle_sparse24_compress.argtypes = [P, i32, i32, P, P]
+        L.oracle_sparse24_decompress.restype = i32
+        L.oracle_sparse24_decompress.argtypes = [P, P, i32, i32, P]
+        L.oracle_quantize_sparse24.restype = i32
+        L.oracle_quantize_sparse24.argtypes = [P, i32, i32, P, P, P, P]
+        L.oracle_gemm_sparse24.restype = i32
+        L.oracle_gemm_sparse24.argtypes = [P, P, P, P, P, f32, i32, i32, i32, P, P, P]
         _lib = L
     return _lib
 
@@ -182,3 +190,56 @@ def swizzle_scales(s: np.ndarray, rows: int, K: int) -> np.ndarray:
 def bf16_bits_to_float(bits: np.ndarray) -> np.ndarray:
     """Widen BF16 bit patterns to fp32 (a bit shift; no rounding involved)."""
     return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- 2:4 sparsity
+# Layout and pruning rule: see oracle_sparse24_* in nvfp4_oracle.h.
+
+def sparse24_compress(codes: np.ndarray, K: int):
+    """Dense packed codes u8 [rows, K/2] with at most 2 non-zero bytes in every
+    4 -> (values u8 [rows, K/4], meta u8 [rows, K/16])."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows = codes.shape[0]
+    values = np.zeros((rows, K // 4), np.uint8)
+    meta = np.zeros((rows, K // 16), np.uint8)
+    if lib().oracle_sparse24_compress(_p(codes), rows, K, _p(values), _p(meta)):
+        raise ValueError("oracle_sparse24_compress: a group has more than 2 non-zero bytes, or a bad shape")
+    return values, meta
+
+
+def sparse24_decompress(values: np.ndarray, meta: np.ndarray, K: int) -> np.ndarray:
+    """(values [rows, K/4], meta [rows, K/16]) -> dense packed codes u8 [rows, K/2]."""
+    values = np.ascontiguousarray(values, dtype=np.uint8)
+    meta = np.ascontiguousarray(meta, dtype=np.uint8)
+    rows = values.shape[0]
+    codes = np.zeros((rows, K // 2), np.uint8)
+    if lib().oracle_sparse24_decompress(_p(values), _p(meta), rows, K, _p(codes)):
+        raise ValueError("oracle_sparse24_decompress: invalid metadata or shape")
+    return codes
+
+
+def quantize_sparse24(X: np.ndarray):
+    """fp32 [rows, K] -> pruned to 2:4 over value pairs and quantized:
+    (values [rows, K/4], meta [rows, K/16], scales [rows, K/16], g)."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    rows, K = X.shape
+    values = np.zeros((rows, K // 4), np.uint8)
+    meta = np.zeros((rows, K // 16), np.uint8)
+    scales = np.zeros((rows, K // 16), np.uint8)
+    g = np.zeros(1, np.float32)
+    if lib().oracle_quantize_sparse24(_p(X), rows, K, _p(values), _p(meta), _p(scales), _p(g)):
+        raise ValueError("oracle_quantize_sparse24 rejected its input")
+    return values, meta, scales, float(g[0])
+
+
+def gemm_sparse24(A, sA, Bv, Bm, sB, alpha: float, M: int, N: int, K: int):
+    """Dense A times 2:4-sparse B: (D bf16 bits [M,N], exact f64 [M,N], |alpha| sum|a b| [M,N])."""
+    A, sA, Bv, Bm, sB = (np.ascontiguousarray(x, dtype=np.uint8) for x in (A, sA, Bv, Bm, sB))
+    D = np.zeros((M, N), np.uint16)
+    ref = np.zeros((M, N), np.float64)
+    ad = np.zeros((M, N), np.float64)
+    rc = lib().oracle_gemm_sparse24(_p(A), _p(sA), _p(Bv), _p(Bm), _p(sB), float(alpha), M, N, K,
+                                    _p(D), _p(ref), _p(ad))
+    if rc:
+        raise ValueError("oracle_gemm_sparse24 rejected its input")
+    return D, ref, ad

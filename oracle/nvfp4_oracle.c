@@ -374,3 +374,126 @@ int oracle_swizzle_scales(const uint8_t* s, int rows, int K, uint8_t* out) {
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* 2:4 structured sparsity over packed bytes                                */
+/* ------------------------------------------------------------------------ */
+
+/* A packed byte (a pair of E2M1 values) is zero when both values are +-0. */
+static int pair_is_zero(uint8_t b) { return (b & 0x77) == 0; }
+
+/* The two positions (0..3) a group of four packed bytes keeps: its non-zero
+ * bytes, then the lowest zero bytes until there are two.  -1 when more than
+ * two are non-zero. */
+static int group_positions(const uint8_t* g4, int* i0, int* i1) {
+    int pos[4], n = 0;
+    for (int i = 0; i < 4; i++)
+        if (!pair_is_zero(g4[i])) pos[n++] = i;
+    if (n > 2) return -1;
+    for (int i = 0; i < 4 && n < 2; i++)
+        if (pair_is_zero(g4[i])) pos[n++] = i;
+    if (pos[0] > pos[1]) { int t = pos[0]; pos[0] = pos[1]; pos[1] = t; }
+    *i0 = pos[0];
+    *i1 = pos[1];
+    return 0;
+}
+
+static void put_group(uint8_t* values, uint8_t* meta, long grp, const uint8_t* g4, int i0, int i1) {
+    values[2 * grp] = g4[i0];
+    values[2 * grp + 1] = g4[i1];
+    uint8_t nib = (uint8_t)(i0 | (i1 << 2));
+    if (grp & 1) meta[grp / 2] = (uint8_t)((meta[grp / 2] & 0x0F) | (nib << 4));
+    else meta[grp / 2] = (uint8_t)((meta[grp / 2] & 0xF0) | nib);
+}
+
+int oracle_sparse24_compress(const uint8_t* codes, int rows, int K, uint8_t* values, uint8_t* meta) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
+    long groups = (long)rows * (K / 8);
+    memset(meta, 0, (size_t)((long)rows * (K / 16)));
+    for (long grp = 0; grp < groups; grp++) {
+        int i0, i1;
+        if (group_positions(codes + 4 * grp, &i0, &i1)) return -1;
+        put_group(values, meta, grp, codes + 4 * grp, i0, i1);
+    }
+    return 0;
+}
+
+int oracle_sparse24_decompress(const uint8_t* values, const uint8_t* meta, int rows, int K, uint8_t* codes) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
+    long groups = (long)rows * (K / 8);
+    for (long grp = 0; grp < groups; grp++) {
+        uint8_t nib = (grp & 1) ? (uint8_t)(meta[grp / 2] >> 4) : (uint8_t)(meta[grp / 2] & 0x0F);
+        int i0 = nib & 3, i1 = (nib >> 2) & 3;
+        if (i0 >= i1) return -1;   /* not a valid position pair */
+        uint8_t* g4 = codes + 4 * grp;
+        g4[0] = g4[1] = g4[2] = g4[3] = 0;
+        g4[i0] = values[2 * grp];
+        g4[i1] = values[2 * grp + 1];
+    }
+    return 0;
+}
+
+/* Pruning: in each group of four value pairs (eight values along K) keep the
+ * two pairs whose larger magnitude is largest (ties to the lower position),
+ * set the others to zero, then quantize the pruned tensor as a dense one.
+ * Each group keeps its largest value, so every 16-value block keeps its
+ * amax: block scales and g are those of the unpruned tensor, and the kept
+ * codes are the dense codes. */
+int oracle_quantize_sparse24(const float* X, int rows, int K,
+                             uint8_t* values, uint8_t* meta, uint8_t* scales, float* g_out) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return -1;
+    for (long i = 0; i < (long)rows * K; i++)
+        if (!isfinite(X[i])) return -1;
+    float* P = (float*)malloc(sizeof(float) * (size_t)((long)rows * K > 0 ? (long)rows * K : 1));
+    int* keep = (int*)malloc(sizeof(int) * (size_t)((long)rows * (K / 8) * 2 + 2));
+    uint8_t* codes = (uint8_t*)malloc((size_t)((long)rows * (K / 2) + 1));
+    if (!P || !keep || !codes) { free(P); free(keep); free(codes); return -1; }
+    long groups = (long)rows * (K / 8);
+    for (long grp = 0; grp < groups; grp++) {
+        const float* x = X + 8 * grp;
+        float key[4];
+        for (int p = 0; p < 4; p++) {
+            float a = fabsf(x[2 * p]), b = fabsf(x[2 * p + 1]);
+            key[p] = a > b ? a : b;
+        }
+        /* the two largest keys; a later position wins only when strictly larger */
+        int first = 0;
+        for (int p = 1; p < 4; p++) if (key[p] > key[first]) first = p;
+        int second = -1;
+        for (int p = 0; p < 4; p++) {
+            if (p == first) continue;
+            if (second < 0 || key[p] > key[second]) second = p;
+        }
+        int i0 = first < second ? first : second, i1 = first < second ? second : first;
+        keep[2 * grp] = i0;
+        keep[2 * grp + 1] = i1;
+        for (int p = 0; p < 4; p++) {
+            int kept = (p == i0 || p == i1);
+            P[8 * grp + 2 * p] = kept ? x[2 * p] : 0.0f;
+            P[8 * grp + 2 * p + 1] = kept ? x[2 * p + 1] : 0.0f;
+        }
+    }
+    int rc = oracle_quantize(P, rows, K, codes, scales, g_out);
+    if (rc == 0) {
+        memset(meta, 0, (size_t)((long)rows * (K / 16)));
+        for (long grp = 0; grp < groups; grp++)
+            put_group(values, meta, grp, codes + 4 * grp, keep[2 * grp], keep[2 * grp + 1]);
+    }
+    free(P);
+    free(keep);
+    free(codes);
+    return rc;
+}
+
+int oracle_gemm_sparse24(const uint8_t* A, const uint8_t* sA,
+                         const uint8_t* Bv, const uint8_t* Bm, const uint8_t* sB,
+                         float alpha, int M, int N, int K,
+                         uint16_t* D_bf16, double* ref, double* absdot) {
+    if (!gemm_args_ok(M, N, K)) return -1;
+    uint8_t* B = (uint8_t*)malloc((size_t)((long)N * (K / 2) + 1));
+    if (!B) return -1;
+    int rc = oracle_sparse24_decompress(Bv, Bm, N, K, B);
+    if (rc == 0) rc = oracle_gemm(A, sA, B, sB, alpha, M, N, K, D_bf16, ref, absdot);
+    free(B);
+    return rc;
+}

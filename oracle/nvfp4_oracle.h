@@ -93,6 +93,43 @@ uint16_t oracle_bf16_of_scaled(int64_t s_hi, uint64_t s_lo, float alpha);
 long oracle_swizzled_bytes(int rows, int K);
 int  oracle_swizzle_scales(const uint8_t* s_rowmajor, int rows, int K, uint8_t* out);
 
+/* 2:4 structured sparsity over packed bytes.  The pages name FP4 structured
+ * sparsity as a way to cut what small-batch decode demands ("Peeling the
+ * Kernel Onion", sections "Assumptions Embedded in the Benchmark" and
+ * "Knowledge Created and Its Impact") and give no layout; the reading here:
+ * in every group of 4 consecutive packed bytes of a row (8 values along K,
+ * the bytes being pairs of E2M1 values 2p, 2p+1) at most 2 bytes are
+ * non-zero.  A row of K values is stored as
+ *   values [K/4]:  the 2 kept bytes of each group, lower position first;
+ *   meta   [K/16]: per group a nibble p0 | p1 << 2 (positions 0..3, p0 < p1),
+ *                  the even group in the low nibble of each byte;
+ *   scales [K/16]: the dense E4M3 block scales, one per 16 values.
+ * A group with fewer than 2 non-zero bytes keeps its non-zero byte (if any)
+ * and the lowest zero bytes.  K must be a multiple of 16.
+ *
+ * compress returns -1 when a group has more than 2 non-zero bytes;
+ * decompress writes dense codes [rows][K/2] (dropped bytes 0x00) and returns
+ * -1 for a position pair that is not p0 < p1.  Parity: pinned by a worked
+ * layout example, round trips, and the pruning quantizer's reduction to the
+ * dense quantizer (tests/test_oracle_sparse24.py). */
+int oracle_sparse24_compress(const uint8_t* codes, int rows, int K, uint8_t* values, uint8_t* meta);
+int oracle_sparse24_decompress(const uint8_t* values, const uint8_t* meta, int rows, int K, uint8_t* codes);
+
+/* Prune fp32 X[rows][K] to the pattern above -- in each group of 4 value
+ * pairs keep the 2 pairs with the largest max(|x_2p|, |x_2p+1|), ties to the
+ * lower position -- and quantize the pruned tensor like oracle_quantize.
+ * Every group keeps its largest value, so block scales and g equal those of
+ * the unpruned tensor and kept codes equal its dense codes. */
+int oracle_quantize_sparse24(const float* X, int rows, int K,
+                             uint8_t* values, uint8_t* meta, uint8_t* scales, float* g_out);
+
+/* D = A (dense) times the 2:4-sparse B (values, meta, scales) transposed:
+ * by definition the dense GEMM of A and the decompressed B. */
+int oracle_gemm_sparse24(const uint8_t* A, const uint8_t* sA,
+                         const uint8_t* Bv, const uint8_t* Bm, const uint8_t* sB,
+                         float alpha, int M, int N, int K,
+                         uint16_t* D_bf16, double* ref, double* absdot);
+
 #ifdef __cplusplus
 }
 #endif
