@@ -74,6 +74,12 @@ def lib():
         L.oracle_quantize_sparse24.restype = i32
         L.oracle_quantize_sparse24.argtypes = [P, i32, i32, P, P, P, P]
         L.oracle_gemm_sparse24.restype = i32
+        L.oracle_e8m0_value.restype = ctypes.c_double
+        L.oracle_e8m0_value.argtypes = [i32]
+        L.oracle_quantize_mxfp4.restype = i32
+        L.oracle_quantize_mxfp4.argtypes = [P, i32, i32, P, P]
+        L.oracle_gemm_mxfp4.restype = i32
+        L.oracle_gemm_mxfp4.argtypes = [P, P, P, P, f32, i32, i32, i32, P, P, P]
         L.oracle_gemm_sparse24.argtypes = [P, P, P, P, P, f32, i32, i32, i32, P, P, P]
         _lib = L
     return _lib
@@ -242,4 +248,33 @@ def gemm_sparse24(A, sA, Bv, Bm, sB, alpha: float, M: int, N: int, K: int):
                                     _p(D), _p(ref), _p(ad))
     if rc:
         raise ValueError("oracle_gemm_sparse24 rejected its input")
+    return D, ref, ad
+
+
+# ---------------------------------------------------------------- MXFP4
+# E2M1 values, one E8M0 scale (2^(byte - 127)) per 32 values: see nvfp4_oracle.h.
+
+def e8m0_value(byte: int) -> float:
+    return lib().oracle_e8m0_value(int(byte))
+
+
+def quantize_mxfp4(X: np.ndarray):
+    """fp32 [rows, K] -> (codes u8 [rows, K/2], E8M0 scales u8 [rows, K/32])."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    rows, K = X.shape
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((rows, K // 32), np.uint8)
+    if lib().oracle_quantize_mxfp4(_p(X), rows, K, _p(codes), _p(scales)):
+        raise ValueError("oracle_quantize_mxfp4 rejected its input")
+    return codes, scales
+
+
+def gemm_mxfp4(A, sA, B, sB, alpha: float, M: int, N: int, K: int):
+    """-> (D bf16 bits [M,N], exact value f64 [M,N], |alpha| sum|a_k b_k| f64 [M,N])."""
+    A, sA, B, sB = (np.ascontiguousarray(x, dtype=np.uint8) for x in (A, sA, B, sB))
+    D = np.zeros((M, N), np.uint16)
+    ref = np.zeros((M, N), np.float64)
+    ad = np.zeros((M, N), np.float64)
+    if lib().oracle_gemm_mxfp4(_p(A), _p(sA), _p(B), _p(sB), float(alpha), M, N, K, _p(D), _p(ref), _p(ad)):
+        raise ValueError("oracle_gemm_mxfp4 rejected its input")
     return D, ref, ad

@@ -497,3 +497,217 @@ int oracle_gemm_sparse24(const uint8_t* A, const uint8_t* sA,
     free(B);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4: E2M1 values, one E8M0 (power of two) scale per 32 values          */
+/* ------------------------------------------------------------------------ */
+
+double oracle_e8m0_value(int byte) {
+    if (byte < 0 || byte > 255) return NAN;
+    if (byte == 255) return NAN;
+    return ldexp(1.0, byte - 127);
+}
+
+/* Per block of 32: X = 2^(floor(log2 amax) - 2) (2 = the exponent of E2M1's
+ * largest value, 6 = 1.5 * 2^2), clamped to 2^-127 .. 2^127 and stored as
+ * the byte log2(X) + 127; codes = E2M1(x / X), nearest even, saturating at 6,
+ * keeping the sign of a value that rounds to zero.  An all-zero block gets
+ * the byte 0 and zero codes. */
+int oracle_quantize_mxfp4(const float* X, int rows, int K, uint8_t* codes, uint8_t* scales) {
+    if (rows < 0 || K <= 0 || K % 32 != 0) return -1;
+    for (long i = 0; i < (long)rows * K; i++)
+        if (!isfinite(X[i])) return -1;
+    for (int r = 0; r < rows; r++) {
+        const float* x = X + (long)r * K;
+        uint8_t* crow = codes + (long)r * (K / 2);
+        memset(crow, 0, (size_t)(K / 2));
+        for (int b = 0; b < K / 32; b++) {
+            float amax = 0.0f;
+            for (int i = 0; i < 32; i++) {
+                float a = fabsf(x[32 * b + i]);
+                if (a > amax) amax = a;
+            }
+            int shared = -127;
+            if (amax > 0.0f) {
+                int e;
+                frexpf(amax, &e);               /* amax = f * 2^e, f in [0.5, 1) */
+                shared = (e - 1) - 2;
+                if (shared < -127) shared = -127;
+                if (shared > 127) shared = 127;
+            }
+            scales[(long)r * (K / 32) + b] = (uint8_t)(amax > 0.0f ? shared + 127 : 0);
+            volatile float Xs = ldexpf(1.0f, shared);
+            for (int i = 0; i < 32; i++) {
+                int k = 32 * b + i;
+                int q;
+                if (amax == 0.0f) {
+                    q = signbit(x[k]) ? 8 : 0;
+                } else {
+                    volatile float v = x[k] / Xs;
+                    q = oracle_e2m1_rne_satfinite(v);
+                }
+                crow[k / 2] |= (uint8_t)((k & 1) ? (q << 4) : q);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Unsigned big integers, 32-bit limbs, little endian: the exact sums of MX
+ * products span 2^-256 .. 2^267 (scales 2^-127 .. 2^127 on each side). */
+#define BIG_LIMBS 24
+typedef struct { uint32_t w[BIG_LIMBS]; } big_t;
+
+static void big_add_shifted(big_t* x, uint64_t v, int shift) {
+    int limb = shift / 32, bit = shift % 32;
+    u128 carry = (u128)v << bit;
+    for (int i = limb; i < BIG_LIMBS && carry; i++) {
+        carry += x->w[i];
+        x->w[i] = (uint32_t)carry;
+        carry >>= 32;
+    }
+}
+
+static int big_cmp(const big_t* a, const big_t* b) {
+    for (int i = BIG_LIMBS - 1; i >= 0; i--)
+        if (a->w[i] != b->w[i]) return a->w[i] < b->w[i] ? -1 : 1;
+    return 0;
+}
+
+static void big_sub(big_t* a, const big_t* b) {   /* a -= b, a >= b */
+    int64_t borrow = 0;
+    for (int i = 0; i < BIG_LIMBS; i++) {
+        int64_t d = (int64_t)a->w[i] - (int64_t)b->w[i] - borrow;
+        borrow = d < 0;
+        a->w[i] = (uint32_t)(d + (borrow ? ((int64_t)1 << 32) : 0));
+    }
+}
+
+static void big_mul_small(big_t* a, uint32_t m) {
+    uint64_t carry = 0;
+    for (int i = 0; i < BIG_LIMBS; i++) {
+        uint64_t t = (uint64_t)a->w[i] * m + carry;
+        a->w[i] = (uint32_t)t;
+        carry = t >> 32;
+    }
+}
+
+static int big_bitlen(const big_t* a) {
+    for (int i = BIG_LIMBS - 1; i >= 0; i--)
+        if (a->w[i]) {
+            int n = 32;
+            while (!(a->w[i] >> (n - 1))) n--;
+            return 32 * i + n;
+        }
+    return 0;
+}
+
+static int big_bit(const big_t* a, int i) { return i < 0 ? 0 : (int)((a->w[i / 32] >> (i % 32)) & 1u); }
+
+static int big_any_below(const big_t* a, int i) {   /* any bit at index < i */
+    for (int j = 0; j < i; j++)
+        if (big_bit(a, j)) return 1;
+    return 0;
+}
+
+static uint64_t big_shr_small(const big_t* a, int s) {   /* a >> s, known to fit 64 bits */
+    uint64_t r = 0;
+    for (int j = 0; j < 64; j++) r |= (uint64_t)big_bit(a, s + j) << j;
+    return r;
+}
+
+/* BF16 (round to nearest even) of sign * P * 2^E, P a big integer. */
+static uint16_t bf16_rne_big(int sign, const big_t* P, int E) {
+    int nb = big_bitlen(P);
+    if (nb == 0) return 0x0000;                 /* an exact zero is reported as +0 */
+    int ev = nb - 1 + E;                        /* 2^ev <= value < 2^(ev+1) */
+    int shift = (ev >= -126) ? nb - 8 : (-133 - E);
+    uint64_t q;
+    if (shift > 0) {
+        q = big_shr_small(P, shift);
+        int half = big_bit(P, shift - 1), sticky = big_any_below(P, shift - 1);
+        if (half && (sticky || (q & 1))) q++;
+    } else {
+        q = big_shr_small(P, 0) << (-shift);
+    }
+    int eq = E + shift;
+    if (q == 256) { q = 128; eq += 1; }
+    uint16_t bits;
+    if (q >= 128) {
+        int biased = eq + 7 + 127;
+        if (biased >= 255) bits = 0x7F80;
+        else bits = (uint16_t)((biased << 7) | (int)(q - 128));
+    } else {
+        bits = (uint16_t)q;
+    }
+    return (uint16_t)((sign << 15) | bits);
+}
+
+static double big_to_double(const big_t* P, int E) {
+    int nb = big_bitlen(P);
+    if (nb == 0) return 0.0;
+    int s = nb > 64 ? nb - 64 : 0;
+    return ldexp((double)big_shr_small(P, s), s + E);
+}
+
+/* One exact MX dot product of K values (K % 32 == 0). */
+static uint16_t mx_dot(const uint8_t* a, const uint8_t* sa, const uint8_t* b, const uint8_t* sb, int K,
+                       float alpha, double* exact, double* absdot) {
+    big_t pos, neg;
+    memset(&pos, 0, sizeof pos);
+    memset(&neg, 0, sizeof neg);
+    double ad = 0.0;
+    for (int blk = 0; blk < K / 32; blk++) {
+        long s = 0, sabs = 0;                   /* quarter units: e2m1 half units squared */
+        for (int i = 0; i < 32; i++) {
+            int k = 32 * blk + i;
+            int ca = (k & 1) ? (a[k / 2] >> 4) : (a[k / 2] & 0xF);
+            int cb = (k & 1) ? (b[k / 2] >> 4) : (b[k / 2] & 0xF);
+            long t = (long)e2m1_half_units(ca) * e2m1_half_units(cb);
+            if ((ca ^ cb) & 8) t = -t;
+            s += t;
+            sabs += t < 0 ? -t : t;
+        }
+        int E = ((int)sa[blk] - 127) + ((int)sb[blk] - 127) - 2;   /* value = s * 2^E */
+        if (s > 0) big_add_shifted(&pos, (uint64_t)s, E + 256);
+        if (s < 0) big_add_shifted(&neg, (uint64_t)(-s), E + 256);
+        ad += ldexp((double)sabs, E);
+    }
+    int sign = 0;
+    if (big_cmp(&pos, &neg) >= 0) {
+        big_sub(&pos, &neg);
+    } else {
+        big_sub(&neg, &pos);
+        pos = neg;
+        sign = 1;
+    }
+    /* alpha = +-ma * 2^ea2 exactly */
+    uint32_t abits;
+    memcpy(&abits, &alpha, 4);
+    int sign_a = (int)(abits >> 31), ea = (int)((abits >> 23) & 0xFF);
+    uint32_t ma = ea ? ((abits & 0x7FFFFF) | 0x800000u) : (abits & 0x7FFFFF);
+    int ea2 = ea ? ea - 150 : -149;
+    double mag = big_to_double(&pos, -256);
+    if (exact) *exact = (sign ? -mag : mag) * (double)alpha;
+    if (absdot) *absdot = ad * fabs((double)alpha);
+    big_mul_small(&pos, ma);
+    return bf16_rne_big(sign ^ sign_a, &pos, -256 + ea2);
+}
+
+int oracle_gemm_mxfp4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
+                      float alpha, int M, int N, int K, uint16_t* D_bf16, double* ref, double* absdot) {
+    if (M < 0 || N < 0 || K <= 0 || K % 32 != 0 || K > (1 << 20) || !isfinite(alpha)) return -1;
+    for (long i = 0; i < (long)M * (K / 32); i++) if (sA[i] == 0xFF) return -1;
+    for (long i = 0; i < (long)N * (K / 32); i++) if (sB[i] == 0xFF) return -1;
+    for (int m = 0; m < M; m++)
+        for (int n = 0; n < N; n++) {
+            double e, ad;
+            uint16_t d = mx_dot(A + (long)m * (K / 2), sA + (long)m * (K / 32), B + (long)n * (K / 2),
+                                sB + (long)n * (K / 32), K, alpha, &e, &ad);
+            long o = (long)m * N + n;
+            if (D_bf16) D_bf16[o] = d;
+            if (ref) ref[o] = e;
+            if (absdot) absdot[o] = ad;
+        }
+    return 0;
+}

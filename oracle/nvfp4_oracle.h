@@ -130,6 +130,27 @@ int oracle_gemm_sparse24(const uint8_t* A, const uint8_t* sA,
                          float alpha, int M, int N, int K,
                          uint16_t* D_bf16, double* ref, double* absdot);
 
+/* MXFP4 (the other block-scaled FP4 format of the same tensor-core
+ * instruction family; the pages do not use it): E2M1 values with one E8M0
+ * scale -- a power of two 2^(byte - 127), byte 255 NaN -- per 32 values
+ * along K, scales [rows][K/32].
+ *   oracle_quantize_mxfp4: per block X = 2^(floor(log2 amax) - 2), clamped to
+ *   2^-127 .. 2^127; codes E2M1(x / X) nearest even, saturating at 6, zero
+ *   codes keep the sign of x; an all-zero block gets scale byte 0 and zero
+ *   codes.  -1 for K % 32 != 0 or a non-finite input.
+ *   oracle_gemm_mxfp4: D = bf16_rne(alpha * sum_k e2m1(A) 2^(sA-127)
+ *   e2m1(B) 2^(sB-127)), the sum exact in a 768-bit integer (products span
+ *   2^-256 .. 2^256), alpha applied exactly, one rounding; ref and absdot as
+ *   for oracle_gemm.  -1 for a NaN scale (255), K % 32 != 0 or a non-finite
+ *   alpha.
+ * Parity: pinned by the E8M0 closed form, hand-worked quantizer blocks, brute
+ * force with exact rationals, and the reduction to oracle_gemm when every
+ * scale is 1 (tests/test_oracle_mxfp4.py). */
+double oracle_e8m0_value(int byte);
+int oracle_quantize_mxfp4(const float* X, int rows, int K, uint8_t* codes, uint8_t* scales);
+int oracle_gemm_mxfp4(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
+                      float alpha, int M, int N, int K, uint16_t* D_bf16, double* ref, double* absdot);
+
 #ifdef __cplusplus
 }
 #endif
