@@ -680,6 +680,79 @@ def run_decode(args):
             "hbm_gbs": hbm_gbs, "shapes": rows}
 
 
+def run_sparse(args):
+    """2:4-sparse weights against dense ones on decode shapes: the same token
+    rows and the same (pruned) weights, once compressed through
+    nvfp4_gemm_sparse24 and once expanded through nvfp4_gemm; graph-replayed
+    back-to-back calls over rotating buffers, us per GEMM."""
+    import torch
+    import nvfp4_block_scaled_gemm_b200 as nv
+    dev = torch.device("cuda", 0)
+    nv.lib()
+    hbm_gbs = load_peaks()[0]
+    stream = torch.cuda.Stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    rows = []
+    for (Nn, Kk) in ((768, 6144), (2048, 6144), (8192, 8192)):
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2300 + Nn)
+        W = torch.randn((Nn, Kk), generator=gen, device=dev) * 0.02
+        # prune on the device with the oracle's rule (keep the 2 pairs of each
+        # 4 with the largest element magnitude), then quantize densely
+        key = W.abs().view(Nn, Kk // 8, 4, 2).amax(dim=3)
+        idx = torch.topk(key, 2, dim=2, largest=True, sorted=False).indices
+        keep = torch.zeros_like(key, dtype=torch.bool).scatter_(2, idx, True)
+        Wp = torch.where(keep.repeat_interleave(2, dim=2).view(Nn, Kk), W, torch.zeros_like(W))
+        cb, sb, gb = nv.quantize(Wp)
+        # compress: kept bytes in position order and their nibbles
+        grp = cb.view(Nn, Kk // 8, 4)
+        pos = torch.sort(idx, dim=2).values
+        bv = torch.gather(grp, 2, pos.to(torch.int64)).reshape(Nn, Kk // 4).contiguous()
+        nib = (pos[..., 0] | (pos[..., 1] << 2)).to(torch.uint8)
+        bm = (nib[:, 0::2] | (nib[:, 1::2] << 4)).contiguous()
+        for M in (1, 2, 4, 8):
+            A32 = torch.randn((M, Kk), generator=gen, device=dev)
+            ca, sa, ga = nv.quantize(A32)
+            alpha = float(ga.item() * gb.item())
+            per_set = Nn * Kk // 2 + Nn * Kk // 16
+            R = int(max(2, min(64, -(-4 * l2 // per_set))))
+            dense_sets = [(cb.clone(), sb.clone(), torch.empty((M, Nn), dtype=torch.bfloat16, device=dev))
+                          for _ in range(R)]
+            sparse_sets = [(bv.clone(), bm.clone(), sb.clone(), torch.empty((M, Nn), dtype=torch.bfloat16, device=dev))
+                           for _ in range(R)]
+
+            def timed(enqueue):
+                with torch.cuda.stream(stream):
+                    enqueue()
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    enqueue()
+                reps = max(1, min(args.steps, 2000) // R)
+                with torch.cuda.stream(stream):
+                    g.replay()
+                stream.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record(stream)
+                stream.synchronize()
+                assert nv.get_device_error(stream) == 0
+                return e0.elapsed_time(e1) * 1e3 / (reps * R)
+
+            us_dense = timed(lambda: [nv.gemm(ca, sa, b, s, alpha, out=o, stream=stream) for (b, s, o) in dense_sets])
+            us_sparse = timed(lambda: [nv.gemm_sparse24(ca, sa, v, m, s, alpha, out=o, stream=stream)
+                                       for (v, m, s, o) in sparse_sets])
+            sparse_bytes = M * Kk // 2 + M * Kk // 16 + Nn * Kk // 4 + 2 * Nn * Kk // 16 + 2 * M * Nn
+            rows.append({"M": M, "N": Nn, "K": Kk, "us_dense": round(us_dense, 2), "us_sparse": round(us_sparse, 2),
+                         "sparse_GBps": round(sparse_bytes / us_sparse / 1e3, 1),
+                         "sparse_hbm_frac": round(sparse_bytes / us_sparse / 1e3 / hbm_gbs, 4)})
+    return {"workload": "2:4-sparse weights vs dense on decode shapes (us per GEMM, graph-replayed back-to-back "
+                        "calls, rotating buffers > 4x L2)", "hbm_gbs": hbm_gbs, "shapes": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -687,7 +760,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain", "pages", "decode"],
+    ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain", "pages", "decode",
+                                           "sparse"],
                     default="attn",
                     help="attn (default) prints the benchmark line; the others print a per-shape report")
     args = ap.parse_args()
@@ -710,6 +784,8 @@ def main():
                 print(json.dumps(run_chain(args)), flush=True)
             elif args.workload == "decode":
                 print(json.dumps(run_decode(args)), flush=True)
+            elif args.workload == "sparse":
+                print(json.dumps(run_sparse(args)), flush=True)
             else:
                 shapes = {"moe": synth.moe_sweep, "pages": synth.pages_sweep}.get(args.workload, synth.saturation_sweep)()
                 print(json.dumps(run_shapes(args, shapes, args.workload)), flush=True)

@@ -278,6 +278,33 @@ nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA,
                                 float alpha, void* D,
                                 int M, int N, int K, void* stream);
 
+/*
+ * nvfp4_gemm_sparse24 -- D = alpha * A * B^T with 2:4-sparse NVFP4 weights B.
+ * The pages name FP4 structured sparsity as a way to cut what small-batch
+ * decode demands ("Peeling the Kernel Onion", sections "Assumptions Embedded
+ * in the Benchmark" and "Knowledge Created and Its Impact") and give no
+ * layout; this library's layout: of every 4 consecutive packed bytes of a
+ * row of B (pairs of E2M1 values) at most 2 are non-zero, stored as
+ *   Bv [N][K/4]:  the 2 kept bytes of each group of 4, lower position first;
+ *   Bm [N][K/16]: per group a nibble p0 | p1 << 2 (positions 0..3, p0 < p1),
+ *                 the even group in the low nibble of each byte;
+ *   sB [N][K/16]: the dense E4M3 block scales, as for nvfp4_gemm.
+ * The result is nvfp4_gemm's on the dense B this describes (dropped bytes
+ * zero).  A, sA, alpha, D and the flags are as for nvfp4_gemm_ex.
+ *   Requirements: K % 64 == 0, N % 8 == 0; A, Bv, D 16-byte aligned; sA, Bm,
+ *   sB 4-byte aligned.  Metadata nibbles with p0 >= p1 are not checked; they
+ *   give an unspecified result but every access stays inside the arguments.
+ *   Up to 8 token rows (NVFP4_GEMM_SP24_GEMV=<n> sets the limit, 0..16) run a
+ *   CUDA-core kernel on the compressed weights, reading 6K/16 weight bytes
+ *   per row instead of 9K/16.  Above it B is expanded to dense codes in
+ *   per-stream scratch (may cudaMalloc on a stream's first use of a size, as
+ *   nvfp4_gemm's scratch) and the dense GEMM runs.
+ */
+nvfp4_status nvfp4_gemm_sparse24(const void* A, const void* sA,
+                                 const void* Bv, const void* Bm, const void* sB,
+                                 float alpha, void* D,
+                                 int M, int N, int K, unsigned flags, void* stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int nvfp4_version(void);
 

@@ -33,6 +33,7 @@ EXPORTS = (
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
     "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe", "nvfp4_quantize_scaled", "nvfp4_gemm_bf16a",
+    "nvfp4_gemm_sparse24",
 )
 
 
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize_scaled.restype = i32
         L.nvfp4_gemm_bf16a.argtypes = [P, f32, P, P, f32, P, i32, i32, i32, P]
         L.nvfp4_gemm_bf16a.restype = i32
+        L.nvfp4_gemm_sparse24.argtypes = [P, P, P, P, P, f32, P, i32, i32, i32, ctypes.c_uint, P]
+        L.nvfp4_gemm_sparse24.restype = i32
         _lib = L
     return _lib
 
@@ -165,6 +168,34 @@ def gemm_noalloc(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.T
     _need(out, "out", torch.bfloat16, (M, N))
     _check(lib().nvfp4_gemm_noalloc(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
                                     out.data_ptr(), M, N, K, _stream(stream)), "nvfp4_gemm_noalloc")
+    return out
+
+
+def gemm_sparse24(A: torch.Tensor, sA: torch.Tensor, Bv: torch.Tensor, Bm: torch.Tensor, sB: torch.Tensor,
+                  alpha: float, out: torch.Tensor | None = None, stream=None,
+                  b_constant: bool = False) -> torch.Tensor:
+    """D[M,N] (bf16) = alpha * (A * sA) @ (B * sB)^T with 2:4-sparse weights.
+
+    A uint8 [M, K/2], sA uint8 [M, K/16]; B as kept bytes Bv uint8 [N, K/4],
+    position nibbles Bm uint8 [N, K/16] and scales sB uint8 [N, K/16] (layout
+    in nvfp4_gemm.h, nvfp4_gemm_sparse24)."""
+    if A.dim() != 2 or Bv.dim() != 2:
+        raise ValueError("A must be [M, K/2] packed codes and Bv [N, K/4] kept bytes")
+    M, N, K = A.shape[0], Bv.shape[0], packed_k(A)
+    if Bv.shape[1] * 4 != K:
+        raise ValueError(f"K mismatch: A holds K={K} (shape {tuple(A.shape)}), Bv holds K={Bv.shape[1] * 4} "
+                         f"(shape {tuple(Bv.shape)}); Bv is [N, K/4]")
+    _need(A, "A", torch.uint8, (M, K // 2))
+    _need(sA, "sA", torch.uint8, (M, K // 16))
+    _need(Bv, "Bv", torch.uint8, (N, K // 4))
+    _need(Bm, "Bm", torch.uint8, (N, K // 16))
+    _need(sB, "sB", torch.uint8, (N, K // 16))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _need(out, "out", torch.bfloat16, (M, N))
+    _check(lib().nvfp4_gemm_sparse24(A.data_ptr(), sA.data_ptr(), Bv.data_ptr(), Bm.data_ptr(), sB.data_ptr(),
+                                     float(alpha), out.data_ptr(), M, N, K, B_CONSTANT if b_constant else 0,
+                                     _stream(stream)), "nvfp4_gemm_sparse24")
     return out
 
 

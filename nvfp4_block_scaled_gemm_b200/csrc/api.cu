@@ -18,6 +18,7 @@
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
 #include "gemv_kernel.cuh"
+#include "sparse_kernel.cuh"
 #include "grouped_kernel.cuh"
 #include "pair_kernel.cuh"
 #include "peak_kernel.cuh"
@@ -536,6 +537,59 @@ nvfp4_status gemv_gemm(DeviceInfo* info, const void* A, const void* sA, const vo
     return launch_gemv_rw<16>(info, rw, prm, stream);
 }
 
+// ---------------------------------------------------- 2:4-sparse weights
+template <int MT, int RW>
+nvfp4_status launch_gemv_sp24_kernel(DeviceInfo* info, const nvfp4::GemvSp24Params& prm, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemv_sp24_kernel<MT, RW>;
+    static const int per_sm = [kern] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, nvfp4::kGemvThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            b = 0;
+        }
+        return b > 0 ? b : 1;
+    }();
+    const int groups = (prm.N + RW - 1) / RW;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(groups, per_sm * info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+template <int MT>
+nvfp4_status launch_gemv_sp24_rw(DeviceInfo* info, int rw, const nvfp4::GemvSp24Params& prm, cudaStream_t stream) {
+    if (rw == 1) return launch_gemv_sp24_kernel<MT, 1>(info, prm, stream);
+    if constexpr (MT <= 2) {
+        if (rw == 4) return launch_gemv_sp24_kernel<MT, 4>(info, prm, stream);
+    }
+    return launch_gemv_sp24_kernel<MT, 2>(info, prm, stream);
+}
+
+// Token rows up to which the 2:4-sparse GEMM runs the CUDA-core kernel on the
+// compressed weights; above it the weights are expanded to dense codes in
+// scratch and the dense GEMM runs.  NVFP4_GEMM_SP24_GEMV=<n> (0..16) moves
+// the limit (tuning and tests).
+int sp24_gemv_max_m() {
+    if (const char* e = std::getenv("NVFP4_GEMM_SP24_GEMV")) {
+        const int v = std::atoi(e);
+        return v < 0 ? 0 : v > 16 ? 16 : v;
+    }
+    return 8;
+}
+
 nvfp4_status launch_pair(DeviceInfo* info, const CUtensorMap& tmA, const CUtensorMap& tmB,
                          const nvfp4::PairParams& prm, cudaStream_t stream) {
     using C = nvfp4::PairConfig;
@@ -1038,6 +1092,77 @@ nvfp4_status nvfp4_fp4_peak_probe(int pair, long long steps, int* ctas_out, void
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// 2:4-sparse weights (nvfp4_gemm_sparse24).
+// ---------------------------------------------------------------------------
+extern "C" nvfp4_status nvfp4_gemm_sparse24(const void* A, const void* sA, const void* Bv, const void* Bm,
+                                            const void* sB, float alpha, void* D, int M, int N, int K,
+                                            unsigned flags, void* stream_) {
+    if (flags & ~NVFP4_GEMM_B_CONSTANT) return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!A || !sA || !Bv || !Bm || !sB || !D) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(Bv, 16) || !aligned(D, 16) || !aligned(sA, 4) || !aligned(sB, 4) ||
+        !aligned(Bm, 4))
+        return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (M <= sp24_gemv_max_m()) {
+        nvfp4::GemvSp24Params prm{};
+        prm.A = static_cast<const uint8_t*>(A);
+        prm.sA = static_cast<const uint8_t*>(sA);
+        prm.Bv = static_cast<const uint8_t*>(Bv);
+        prm.Bm = static_cast<const uint8_t*>(Bm);
+        prm.sB = static_cast<const uint8_t*>(sB);
+        prm.D = static_cast<__nv_bfloat16*>(D);
+        prm.alpha = alpha;
+        prm.M = M;
+        prm.N = N;
+        prm.K = K;
+        prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+        int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
+        if (const char* e = std::getenv("NVFP4_GEMM_GEMV_RW")) {
+            const int v = std::atoi(e);
+            if (v == 1 || v == 2 || v == 4) rw = v;
+        }
+        if (M <= 1) return launch_gemv_sp24_rw<1>(info, rw, prm, stream);
+        if (M <= 2) return launch_gemv_sp24_rw<2>(info, rw, prm, stream);
+        if (M <= 4) return launch_gemv_sp24_rw<4>(info, rw, prm, stream);
+        if (M <= 8) return launch_gemv_sp24_rw<8>(info, rw, prm, stream);
+        return launch_gemv_sp24_rw<16>(info, rw, prm, stream);
+    }
+    // Dense codes in the operand scratch (ordered on the stream before the
+    // GEMM that reads them; the GEMM gets no constant-B flag, since its B is
+    // written right before it).
+    const size_t dense_bytes = (size_t)N * (size_t)(K / 2);
+    uint8_t* dense = nullptr;
+    if ((st = get_scratch(dev, stream, dense_bytes, &dense, /*act=*/true)) != NVFP4_OK) return st;
+    const long long items = (long long)N * (K / 16);
+    const int threads = 256;
+    const int blocks = (int)std::min<long long>((items + threads - 1) / threads, (long long)info->num_sms * 8);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::max(blocks, 1), 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4::sparse24_expand_kernel, static_cast<const uint8_t*>(Bv),
+                                             static_cast<const uint8_t*>(Bm), items, dense);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return nvfp4_gemm_ex(A, sA, dense, sB, alpha, D, M, N, K, 0u, stream_);
+}
 
 // ---------------------------------------------------------------------------
 // GEMM without any device allocation (nvfp4_gemm_noalloc).
