@@ -14,11 +14,13 @@
 //
 // The decode kernel follows nvfp4_gemv_kernel (gemv_kernel.cuh): a thread
 // owns 32-value chunks of K, which here are 8 value bytes, 2 metadata bytes
-// and 2 scale bytes per weight row; each group's two kept pairs meet the
-// activation pairs at the same positions (selected from the decoded chunk),
-// so a 16-value block is 4 fma.rn.f16x2 (8 products per half at most 144 in
-// magnitude: exact), and the rest -- exact block sum times sA * sB, fp32 sum
-// over blocks, warp butterfly, fixed-order CTA sum -- is the dense kernel's.
+// and 2 scale bytes per weight row.  One byte permute per two groups gathers
+// the activation bytes at the kept positions next to the kept weight bytes
+// (its selector built once per weight row and chunk from the metadata), so
+// only kept pairs are decoded and multiplied: a 16-value block is 4
+// fma.rn.f16x2 (4 products per half, at most 144 in magnitude: exact), and
+// the rest -- exact block sum times sA * sB, fp32 sum over blocks, warp
+// butterfly, fixed-order CTA sum -- is the dense kernel's.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -46,13 +48,13 @@ __device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
     return v;
 }
 
-// h4[p] for p in 0..3, without indexing registers at run time.
-__device__ __forceinline__ uint32_t select4(const uint32_t* h4, uint32_t p) {
-    uint32_t x = h4[0];
-    x = p == 1u ? h4[1] : x;
-    x = p == 2u ? h4[2] : x;
-    x = p == 3u ? h4[3] : x;
-    return x;
+// Byte-permute selector that gathers, from two 4-byte activation groups
+// (first group bytes 0..3, second 4..7), the bytes at the kept positions of
+// one metadata byte (low nibble: first group's p0 | p1 << 2, high nibble: the
+// second group's): each 2-bit position becomes a selector nibble, the second
+// group's offset by 4.
+__device__ __forceinline__ uint32_t gather_selector(uint32_t m) {
+    return (m & 0x3u) | ((m & 0xCu) << 2) | ((m & 0x30u) << 4) | ((m & 0xC0u) << 6) | 0x4400u;
 }
 
 template <int MT, int RW>
@@ -128,8 +130,11 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_sp24_kernel(const Gem
                 // kept weight pairs, decoded: bh[r][2j], bh[r][2j+1] for group j
                 uint32_t bh[RW][8];
                 float sb0[RW], sb1[RW];
+                uint32_t sel01[RW], sel23[RW];
 #pragma unroll
                 for (int r = 0; r < RW; ++r) {
+                    sel01[r] = gather_selector(bm[g][r] & 0xFFu);
+                    sel23[r] = gather_selector((bm[g][r] >> 8) & 0xFFu);
                     uint32_t h4[4];
                     e2m1x8_to_f16x2(bq[g][r].x, h4);
                     bh[r][0] = h4[0], bh[r][1] = h4[1], bh[r][2] = h4[2], bh[r][3] = h4[3];
@@ -143,28 +148,32 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_sp24_kernel(const Gem
                     if (m < M) {
                         const uint4 aq = ld_cached_v4(prm.A + (size_t)m * arow_bytes + 16 * (size_t)c);
                         const uint32_t as = ld_cached_u16(prm.sA + (size_t)m * srow_bytes + 2 * (size_t)c);
-                        uint32_t ah[16];
-                        decode_chunk(aq, ah);
                         const float sa0 = e4m3_value(as & 0xFFu), sa1 = e4m3_value(as >> 8);
 #pragma unroll
                         for (int r = 0; r < RW; ++r) {
-                            const uint32_t meta = bm[g][r];
-                            __half2 s[2];
+                            // the activation bytes at the kept positions, in the
+                            // order of the kept weight bytes: groups 0, 1 from
+                            // words x, y; groups 2, 3 from z, w
+                            uint32_t ah[8], t4[4];
+                            e2m1x8_to_f16x2(__byte_perm(aq.x, aq.y, sel01[r]), t4);
+                            ah[0] = t4[0], ah[1] = t4[1], ah[2] = t4[2], ah[3] = t4[3];
+                            e2m1x8_to_f16x2(__byte_perm(aq.z, aq.w, sel23[r]), t4);
+                            ah[4] = t4[0], ah[5] = t4[1], ah[6] = t4[2], ah[7] = t4[3];
+                            float bsum[2];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const uint32_t nib = (meta >> (4 * j)) & 0xFu;
-                                const uint32_t a0 = select4(ah + 4 * j, nib & 3u);
-                                const uint32_t a1 = select4(ah + 4 * j, nib >> 2);
-                                const __half2 p0 = *reinterpret_cast<const __half2*>(&a0);
-                                const __half2 p1 = *reinterpret_cast<const __half2*>(&a1);
-                                const __half2 w0 = *reinterpret_cast<const __half2*>(&bh[r][2 * j]);
-                                const __half2 w1 = *reinterpret_cast<const __half2*>(&bh[r][2 * j + 1]);
-                                if ((j & 1) == 0) s[j >> 1] = __hmul2(p0, w0);
-                                else s[j >> 1] = __hfma2(p0, w0, s[j >> 1]);
-                                s[j >> 1] = __hfma2(p1, w1, s[j >> 1]);
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t* a = ah + 4 * h;
+                                const uint32_t* w = bh[r] + 4 * h;
+                                __half2 s2 = __hmul2(*reinterpret_cast<const __half2*>(&a[0]),
+                                                     *reinterpret_cast<const __half2*>(&w[0]));
+#pragma unroll
+                                for (int i = 1; i < 4; ++i)
+                                    s2 = __hfma2(*reinterpret_cast<const __half2*>(&a[i]),
+                                                 *reinterpret_cast<const __half2*>(&w[i]), s2);
+                                bsum[h] = __low2float(s2) + __high2float(s2);
                             }
-                            acc[r][m] = fmaf(__low2float(s[0]) + __high2float(s[0]), sa0 * sb0[r], acc[r][m]);
-                            acc[r][m] = fmaf(__low2float(s[1]) + __high2float(s[1]), sa1 * sb1[r], acc[r][m]);
+                            acc[r][m] = fmaf(bsum[0], sa0 * sb0[r], acc[r][m]);
+                            acc[r][m] = fmaf(bsum[1], sa1 * sb1[r], acc[r][m]);
                         }
                     }
                 }
