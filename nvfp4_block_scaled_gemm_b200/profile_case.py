@@ -5,10 +5,11 @@
 
 `--traffic-csv FILE` (no GPU) instead turns the CSV log of an ncu run of
 `--shapes attn --iters 2` with the metrics gpu__time_duration.sum,
-dram__bytes_read.sum and dram__bytes_write.sum on the GEMM kernel into the
-per-launch DRAM summary that bench.py reports as `roofline.traffic`
-(profiles/traffic_attn_sweep.json), stamped with the hash of the kernel
-sources it was taken on.
+dram__bytes_read.sum and dram__bytes_write.sum on the GEMM kernels
+(nvfp4_gemm_kernel, and nvfp4_gemv_kernel for M = 1) into the per-launch DRAM
+summary that bench.py reports as `roofline.traffic`
+(profiles/traffic_attn_sweep.json), stamped with the hash of the kernel code
+it was taken on.
 
 `attn` expands to the attention-projection sweep (M in {1,16,64,128,256,512},
 N=768, K=6144).  Inputs are seeded N(0,1) fp32 quantised on the GPU; every
