@@ -259,15 +259,27 @@ nvfp4_status nvfp4_fp4_peak_probe(int pair, long long steps, int* ctas_out, void
  * cudaMalloc scratch on its first call of a new shape; this entry point never
  * calls cudaMalloc, cudaFree or any allocating routine.  It has no counterpart
  * on the source pages; it is a deployment convenience of this library.
- *   Its one piece of scratch -- the operands' scales re-laid out for the
- *   tensor cores -- is a static device array of 8 MiB (8,388,608 bytes) that
- *   every GPU which loads the library keeps until the process exits.  Problems whose scales
- *   need more, i.e. (ceil(M/128) + ceil(N/128)) * (K/64) * 512 bytes (plus up
- *   to 255 bytes of alignment) above that limit, are rejected with
- *   NVFP4_ERR_UNSUPPORTED_SHAPE before anything is launched.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before capturing the stream into a CUDA graph.
+ *   Its scratch is a static device array of 8 MiB (8,388,608 bytes) that
+ *   every GPU which loads the library keeps until the process exits.  A few
+ *   token rows run on the CUDA cores and use none of it.  When K % 256 == 0
+ *   and sA, sB are 16-byte aligned the tensor-core kernels read the
+ *   row-major scales directly, and the array holds at most the fp32 partial
+ *   tiles of a K split (problems large enough for nvfp4_gemm's CTA-pair
+ *   kernel run on the single-CTA persistent kernel instead, as that kernel
+ *   wants its scales re-laid out first).  The other problems (K % 256 != 0,
+ *   or scales only 4-byte aligned) first have their scales re-laid out for
+ *   the tensor cores into the array; such a problem whose scales need more,
+ *   i.e. (ceil(M/128) + ceil(N/128)) * (K/64) * 512 bytes (plus up to 255
+ *   bytes of alignment), is rejected with NVFP4_ERR_UNSUPPORTED_SHAPE before
+ *   anything is launched.  Partial tiles that do not fit after the scales
+ *   make the call run without a K split instead (slower, same result within
+ *   the bound).
+ *   The first call on a device that uses the array looks up its device
+ *   address (cudaGetSymbolAddress, with that device current) and keeps it
+ *   for the life of the process; make that first call before capturing the
+ *   stream into a CUDA graph.  The kept address does not survive
+ *   cudaDeviceReset (which unloads the library's device code): do not call
+ *   this entry point on a device after resetting it.
  *   All calls share the one array, so calls whose work overlaps on the GPU
  *   (different streams, or different host threads) race on it: serialise
  *   them.  Each call rewrites every scratch byte it reads, so no clearing is

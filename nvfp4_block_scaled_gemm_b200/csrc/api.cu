@@ -23,6 +23,7 @@
 #include "pair_kernel.cuh"
 #include "peak_kernel.cuh"
 #include "persistent_kernel.cuh"
+#include "splitk_kernel.cuh"
 
 namespace {
 
@@ -77,12 +78,14 @@ struct Scratch {
     uint8_t* ptr = nullptr;
     size_t cap = 0;
 };
-std::map<std::pair<int, uintptr_t>, Scratch> g_scratch;
-std::map<std::pair<int, uintptr_t>, Scratch> g_act_scratch;   // quantized activations (nvfp4_gemm_bf16a)
+// Kinds of per-(device, stream) scratch, each its own buffer because one call
+// may need several at once.
+enum ScratchKind { kScratchScales = 0, kScratchAct = 1, kScratchSplitK = 2 };
+std::map<std::pair<int, uintptr_t>, Scratch> g_scratch[3];
 
-nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** out, bool act = false) {
+nvfp4_status get_scratch(int dev, cudaStream_t stream, size_t bytes, uint8_t** out, int kind = kScratchScales) {
     std::lock_guard<std::mutex> lk(g_mu);
-    Scratch& s = (act ? g_act_scratch : g_scratch)[{dev, reinterpret_cast<uintptr_t>(stream)}];
+    Scratch& s = g_scratch[kind][{dev, reinterpret_cast<uintptr_t>(stream)}];
     if (s.cap < bytes) {
         size_t want = std::max(bytes, s.cap * 2);
         want = (want + 0xFFFFF) & ~size_t(0xFFFFF);
@@ -290,7 +293,7 @@ int split_cluster_capacity_of(DeviceInfo* info, bool swap, int bq, bool sfr, int
                : split_cluster_capacity_bq<false, false>(info, bq, splits);
 }
 
-Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr) {
+Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr, int max_splits = 8) {
     const int num_sms = info->num_sms;
     Plan p{};
     p.k_tiles = (K + 255) / 256;
@@ -332,10 +335,33 @@ Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr) {
     const int tiles = p.tiles_p * p.tiles_q;
     const int cap = std::min(num_sms, 128);
     int splits = 1;
-    for (int s = 2; s <= 8 && s <= p.k_tiles && tiles * s <= cap; s *= 2)
+    for (int s = 2; s <= max_splits && s <= p.k_tiles && tiles * s <= cap; s *= 2)
         if (split_cluster_capacity_of(info, p.swap, p.bq, sfr, s) >= tiles) splits = s;
     p.splits = splits;
     return p;
+}
+
+// Split-K workspace of a plan: one fp32 partial tile per (tile, rank).
+size_t splitk_ws_bytes(const Plan& p) {
+    return p.splits > 1 ? (size_t)p.tiles_p * p.tiles_q * p.splits * (size_t)p.bq * 128u * 4u : 0;
+}
+
+// The workspace: per-stream scratch (allocated on a stream's first need of
+// that size), or, when `fixed` is given, that caller-owned region of
+// `fixed_cap` bytes (no allocation; too small -> UNSUPPORTED_SHAPE).
+nvfp4_status splitk_ws(int dev, cudaStream_t stream, const Plan& p, uint8_t* fixed, size_t fixed_cap, float4** out) {
+    *out = nullptr;
+    const size_t bytes = splitk_ws_bytes(p);
+    if (bytes == 0) return NVFP4_OK;
+    if (fixed != nullptr) {
+        if (bytes > fixed_cap) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        *out = reinterpret_cast<float4*>(fixed);
+        return NVFP4_OK;
+    }
+    uint8_t* ptr = nullptr;
+    const nvfp4_status st = get_scratch(dev, stream, bytes, &ptr, kScratchSplitK);
+    *out = reinterpret_cast<float4*>(ptr);
+    return st;
 }
 
 struct Maps {
@@ -692,6 +718,258 @@ nvfp4_status launch_mode(const Plan& plan, DeviceInfo* info, const Maps& m, cons
                            : launch_by_bq<false, false, SFR>(plan.bq, info, m, prm, grid, stream);
 }
 
+// ------------------------------------------------- split-K kernel for few token rows
+// Plan of nvfp4_gemm_splitk_kernel: weights in 128-row tiles against the
+// token rows (swapped, M <= 64), or token rows in 128-row tiles against 64-
+// or 128-row weight tiles; K split over a cluster of up to 16 CTAs; every
+// CTA small enough to share its SM with a CTA of the next launch.
+struct SkPlan {
+    bool use = false;
+    bool swap = false;
+    int bq = 0, splits = 1, stages = 1, tiles_p = 0, tiles_q = 0;
+    int smem = 0;
+    uint32_t tmem_cols = 32;
+};
+
+// Two CTAs of at most this much dynamic shared memory fit an SM (228 KB, less
+// 1 KB reserved per CTA); a CTA above kSkSoloSmem has its SM to itself.
+constexpr int kSkCoresidentSmem = 115712;
+constexpr int kSkSoloSmem = 118784;
+
+template <int BQ>
+void sk_fill(SkPlan& p, int nkt, int max_stages) {
+    using C = nvfp4::SkConfig<BQ>;
+    const bool split = p.splits > 1;
+    const int want = std::min({nkt, nvfp4::kSkMaxStages, max_stages});
+    // Co-resident: the whole K slice in a ring that leaves room for a CTA of
+    // the next launch.  Otherwise the deepest ring that fits (the SM to this
+    // CTA): a ring shallower than the K slice is bound by its round trips.
+    int stages = want;
+    while (stages > 1 && nvfp4::sk_smem_bytes<BQ>(stages, split) > kSkCoresidentSmem) --stages;
+    bool solo = false;
+    if (stages < want) {
+        int deep = want;
+        while (deep > 1 && nvfp4::sk_smem_bytes<BQ>(deep, split) > nvfp4::kSmemLimit) --deep;
+        if (deep > stages) {
+            stages = deep;
+            solo = true;
+        }
+    }
+    p.stages = std::max(1, stages);
+    p.smem = nvfp4::sk_smem_bytes<BQ>(p.stages, split);
+    const int cols = C::ACC_COLS + p.stages * C::SF_STRIDE;
+    p.tmem_cols = cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
+    // More than half of TMEM, or a deep ring: keep the SM to this CTA (a
+    // second CTA's TMEM allocation would wait for the first to finish).
+    if (solo || p.tmem_cols > 256) p.smem = std::max(p.smem, kSkSoloSmem);
+}
+
+// The plan: swapped tiles up to 64 token rows; above that 128 token rows
+// against 64 weight rows.  K is split so that the CTAs all run at once, and
+// little enough that the fp32 partials exchanged (splits x M x N x 4 bytes)
+// stay near the size of the weights (N x K / 2 bytes).
+// NVFP4_GEMM_SK=0 turns the kernel off; NVFP4_GEMM_SK="swap:bq:splits:stages"
+// forces a plan where it runs (tuning and tests).
+SkPlan make_sk_plan(int M, int N, int K, const DeviceInfo* info) {
+    SkPlan p;
+    int f_swap = -1, f_bq = 0, f_splits = 0, f_stages = 0;
+    if (const char* e = std::getenv("NVFP4_GEMM_SK")) {
+        if (e[0] == '0' && e[1] == '\0') return p;
+        int a = 0, b = 0, c = 0, d = 0;
+        if (std::sscanf(e, "%d:%d:%d:%d", &a, &b, &c, &d) == 4 && (c == 1 || c == 2 || c == 4 || c == 8 || c == 16) &&
+            d >= 1 && d <= nvfp4::kSkMaxStages &&
+            ((a == 1 && (b == 16 || b == 32 || b == 64)) || (a == 0 && (b == 64 || b == 128)))) {
+            f_swap = a;
+            f_bq = b;
+            f_splits = c;
+            f_stages = d;
+        }
+    }
+    // Measured against the tiled split-K kernel (graph-replayed back-to-back
+    // calls, constant weights): this kernel is faster up to 16 token rows
+    // (768 x 6144: 5.3 against 6.1 us; 2048 x 6144: 6.9 against 7.8;
+    // 256 x 6144: 4.5 against 5.7) and for 64 rows against 256 weight rows;
+    // beyond that the tiled kernel's deeper K pipeline wins.
+    if (f_swap < 0 && !(M <= 16 || (M <= 64 && N <= 256))) return p;
+    const int k_tiles = K / 256;
+    p.swap = f_swap >= 0 ? f_swap == 1 : M <= 64;
+    if (p.swap) {
+        p.bq = f_bq ? f_bq : (M <= 16 ? 16 : 32);
+        p.tiles_p = (N + 127) / 128;
+        p.tiles_q = (M + p.bq - 1) / p.bq;
+    } else {
+        p.bq = f_bq ? f_bq : 64;
+        p.tiles_p = (M + 127) / 128;
+        p.tiles_q = (N + p.bq - 1) / p.bq;
+    }
+    const int tiles = p.tiles_p * p.tiles_q;
+    if (tiles > info->num_sms) return p;   // enough tiles without splitting K: the other kernels
+    const int max_stages = f_stages ? f_stages : nvfp4::kSkMaxStages;
+    auto fill = [&](int splits) {
+        p.splits = splits;
+        const int nkt = (k_tiles + splits - 1) / splits;
+        switch (p.bq) {
+            case 16: sk_fill<16>(p, nkt, max_stages); break;
+            case 32: sk_fill<32>(p, nkt, max_stages); break;
+            case 64: sk_fill<64>(p, nkt, max_stages); break;
+            default: sk_fill<128>(p, nkt, max_stages); break;
+        }
+    };
+    if (f_splits) {
+        int splits = std::min(f_splits, std::max(1, k_tiles));
+        while (splits > 1 && 128 % splits != 0) splits /= 2;
+        fill(splits);
+    } else {
+        // The largest split (a power of two up to 16, at most one per K tile)
+        // whose CTAs all run at once -- two per SM when they are small enough
+        // to share one, else one -- and whose fp32 partials stay within twice
+        // the weight bytes.
+        int splits = 16;
+        for (; splits > 1; splits /= 2) {
+            if (splits > k_tiles || (long long)splits * M * 8 > 2LL * K) continue;
+            fill(splits);
+            const int per_sm = p.smem <= kSkCoresidentSmem ? 2 : 1;
+            if (tiles * splits <= per_sm * info->num_sms) break;
+        }
+        if (splits == 1) fill(1);
+    }
+    p.use = true;
+    return p;
+}
+
+template <int BQ, bool SWAP>
+nvfp4_status launch_sk_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, const nvfp4::SkParams& prm,
+                              const SkPlan& plan, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemm_splitk_kernel<BQ, SWAP>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(info->smem_attr_set & bit)) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, nvfp4::kSmemLimit) !=
+                    cudaSuccess ||
+                cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+                cudaGetLastError();
+                return NVFP4_ERR_CUDA;
+            }
+            info->smem_attr_set |= bit;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)plan.splits, (unsigned)(plan.tiles_p * plan.tiles_q), 1);
+    cfg.blockDim = dim3(nvfp4::kSkThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)plan.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (plan.splits > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)plan.splits;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, m.p, m.q, m.sp, m.sq, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+nvfp4_status sk_gemm(DeviceInfo* info, const SkPlan& plan, const void* A, const void* sA, const void* B,
+                     const void* sB, float alpha, void* D, int M, int N, int K, unsigned flags, cudaStream_t stream) {
+    const void* P = plan.swap ? B : A;
+    const void* Q = plan.swap ? A : B;
+    const void* sP = plan.swap ? sB : sA;
+    const void* sQ = plan.swap ? sA : sB;
+    const int rows_p = plan.swap ? N : M;
+    const int rows_q = plan.swap ? M : N;
+    Maps maps;
+    if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq) ||
+        !make_scale_map(&maps.sp, sP, rows_p, K / 16, 128) || !make_scale_map(&maps.sq, sQ, rows_q, K / 16, plan.bq))
+        return NVFP4_ERR_CUDA;
+    nvfp4::SkParams prm{};
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.alpha = alpha;
+    prm.rows_p = rows_p;
+    prm.rows_q = rows_q;
+    prm.ldd = N;
+    prm.k_tiles = K / 256;
+    prm.tiles_q = plan.tiles_q;
+    prm.stages = plan.stages;
+    prm.prefetch_w = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+    prm.tmem_cols = plan.tmem_cols;
+    if (plan.swap) {
+        switch (plan.bq) {
+            case 16: return launch_sk_kernel<16, true>(info, 1ull << 50, maps, prm, plan, stream);
+            case 32: return launch_sk_kernel<32, true>(info, 1ull << 51, maps, prm, plan, stream);
+            default: return launch_sk_kernel<64, true>(info, 1ull << 52, maps, prm, plan, stream);
+        }
+    }
+    return plan.bq == 64 ? launch_sk_kernel<64, false>(info, 1ull << 54, maps, prm, plan, stream)
+                         : launch_sk_kernel<128, false>(info, 1ull << 53, maps, prm, plan, stream);
+}
+
+// The tensor-core GEMM with row-major scale tiles loaded by TMA (K % 256 == 0,
+// scales 16-byte aligned).  Few token rows take the split-K kernel, large
+// problems the single-CTA persistent kernel, the others the tiled kernel of
+// the plan, whose split-K partials need a workspace: per-stream scratch, or
+// with `ws_fixed` that caller-owned region (when the plan's workspace does
+// not fit it, the plan is made again without a K split).
+nvfp4_status sfr_gemm(int dev, DeviceInfo* info, Plan plan, const void* A, const void* sA, const void* B,
+                      const void* sB, float alpha, void* D, int M, int N, int K, unsigned flags,
+                      cudaStream_t stream, uint8_t* ws_fixed = nullptr, size_t ws_cap = 0) {
+    if (!plan_override().set) {
+        const SkPlan sk = make_sk_plan(M, N, K, info);
+        if (sk.use) return sk_gemm(info, sk, A, sA, B, sB, alpha, D, M, N, K, flags, stream);
+    }
+    if (ws_fixed != nullptr && splitk_ws_bytes(plan) > ws_cap) plan = make_plan(M, N, K, info, true, 1);
+    const void* P = plan.swap ? B : A;
+    const void* Q = plan.swap ? A : B;
+    const void* sP = plan.swap ? sB : sA;
+    const void* sQ = plan.swap ? sA : sB;
+    const int rows_p = plan.swap ? N : M;
+    const int rows_q = plan.swap ? M : N;
+    Maps maps;
+    if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq) ||
+        !make_scale_map(&maps.sp, sP, rows_p, K / 16, 128) || !make_scale_map(&maps.sq, sQ, rows_q, K / 16, plan.bq))
+        return NVFP4_ERR_CUDA;
+    const int tiles = plan.tiles_p * plan.tiles_q;
+    if (!plan.swap && plan.splits == 1 && tiles > info->num_sms && (plan.bq == 128 || plan.bq == 256) &&
+        !plan_override().set) {
+        nvfp4::PersistParams pp{};
+        pp.D = static_cast<__nv_bfloat16*>(D);
+        pp.alpha = alpha;
+        pp.M = M;
+        pp.N = N;
+        pp.K = K;
+        pp.k_tiles = K / 256;
+        pp.tiles_m = plan.tiles_p;
+        pp.tiles_n = plan.tiles_q;
+        return plan.bq == 256 ? launch_persistent<256>(info, 1ull << 60, maps, pp, tiles, stream)
+                              : launch_persistent<128>(info, 1ull << 61, maps, pp, tiles, stream);
+    }
+    GemmParams prm{};
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.alpha = alpha;
+    prm.rows_p = rows_p;
+    prm.rows_q = rows_q;
+    prm.K = K;
+    prm.ldd = N;
+    prm.k_tiles = plan.k_tiles;
+    prm.tiles_q = plan.tiles_q;
+    prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+    nvfp4_status st = splitk_ws(dev, stream, plan, ws_fixed, ws_cap, &prm.ws);
+    if (st != NVFP4_OK) return st;
+    const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
+    return launch_mode<true>(plan, info, maps, prm, grid, stream);
+}
+
 nvfp4_status check_gemm_args(const void* A, const void* sA, const void* B, const void* sB, const void* D, int M,
                              int N, int K) {
     if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
@@ -803,39 +1081,30 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
         2 * ((M + 127) / 128) * ((N + 255) / 256) >= info->num_sms && pair_kernel_enabled() &&
         !plan_override().set)
         return pair_gemm(dev, info, A, sA, B, sB, alpha, D, M, N, K, stream);
+    if (sfr) return sfr_gemm(dev, info, plan, A, sA, B, sB, alpha, D, M, N, K, flags, stream);
+
+    // Scales re-laid out into tensor-core atoms in per-stream scratch.
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
     const void* sP = plan.swap ? sB : sA;
     const void* sQ = plan.swap ? sA : sB;
     const int rows_p = plan.swap ? N : M;
     const int rows_q = plan.swap ? M : N;
-
-    const size_t sfp_bytes = sfr ? 0 : nvfp4_swizzled_scale_bytes(rows_p, K);
-    const size_t sfq_bytes = sfr ? 0 : nvfp4_swizzled_scale_bytes(rows_q, K);
-    const size_t off_sfp = 0;
-    const size_t off_sfq = align_up(off_sfp + sfp_bytes, 256);
+    const size_t sfp_bytes = nvfp4_swizzled_scale_bytes(rows_p, K);
+    const size_t sfq_bytes = nvfp4_swizzled_scale_bytes(rows_q, K);
+    const size_t off_sfq = align_up(sfp_bytes, 256);
     uint8_t* ws = nullptr;
-    if (!sfr) {
-        st = get_scratch(dev, stream, off_sfq + sfq_bytes, &ws);
-        if (st != NVFP4_OK) return st;
-    }
-
+    if ((st = get_scratch(dev, stream, off_sfq + sfq_bytes, &ws)) != NVFP4_OK) return st;
     Maps maps;
     if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq))
         return NVFP4_ERR_CUDA;
-    if (sfr) {
-        if (!make_scale_map(&maps.sp, sP, rows_p, K / 16, 128) || !make_scale_map(&maps.sq, sQ, rows_q, K / 16, plan.bq))
-            return NVFP4_ERR_CUDA;
-    } else {
-        if ((st = launch_swizzle(sP, rows_p, K, ws + off_sfp, stream)) != NVFP4_OK) return st;
-        if ((st = launch_swizzle(sQ, rows_q, K, ws + off_sfq, stream)) != NVFP4_OK) return st;
-        maps.sp = maps.p;
-        maps.sq = maps.q;
-    }
-
+    if ((st = launch_swizzle(sP, rows_p, K, ws, stream)) != NVFP4_OK) return st;
+    if ((st = launch_swizzle(sQ, rows_q, K, ws + off_sfq, stream)) != NVFP4_OK) return st;
+    maps.sp = maps.p;
+    maps.sq = maps.q;
     GemmParams prm{};
-    prm.sfp = sfr ? nullptr : ws + off_sfp;
-    prm.sfq = sfr ? nullptr : ws + off_sfq;
+    prm.sfp = ws;
+    prm.sfq = ws + off_sfq;
     prm.D = static_cast<__nv_bfloat16*>(D);
     prm.alpha = alpha;
     prm.rows_p = rows_p;
@@ -844,26 +1113,10 @@ nvfp4_status nvfp4_gemm_ex(const void* A, const void* sA, const void* B, const v
     prm.ldd = N;
     prm.k_tiles = plan.k_tiles;
     prm.tiles_q = plan.tiles_q;
-    prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
-    // More tiles than SMs, no split, row-major scales: the persistent kernel.
-    const int tiles = plan.tiles_p * plan.tiles_q;
-    if (sfr && !plan.swap && plan.splits == 1 && tiles > info->num_sms && (plan.bq == 128 || plan.bq == 256) &&
-        !plan_override().set) {
-        nvfp4::PersistParams pp{};
-        pp.D = static_cast<__nv_bfloat16*>(D);
-        pp.alpha = alpha;
-        pp.M = M;
-        pp.N = N;
-        pp.K = K;
-        pp.k_tiles = K / 256;
-        pp.tiles_m = plan.tiles_p;
-        pp.tiles_n = plan.tiles_q;
-        return plan.bq == 256 ? launch_persistent<256>(info, 1ull << 60, maps, pp, tiles, stream)
-                              : launch_persistent<128>(info, 1ull << 61, maps, pp, tiles, stream);
-    }
+    prm.prefetch_b = 0;   // the early prefetch reads row-major scale tiles only
+    if ((st = splitk_ws(dev, stream, plan, nullptr, 0, &prm.ws)) != NVFP4_OK) return st;
     const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
-    return sfr ? launch_mode<true>(plan, info, maps, prm, grid, stream)
-               : launch_mode<false>(plan, info, maps, prm, grid, stream);
+    return launch_mode<false>(plan, info, maps, prm, grid, stream);
 }
 
 nvfp4_status nvfp4_grouped_gemm(const void* A, const void* sA, const void* B, const void* sB, const float* alpha,
@@ -1031,6 +1284,7 @@ nvfp4_status nvfp4_gemm_bf16a(const void* A, float gA, const void* B, const void
         prm.k_tiles = plan.k_tiles;
         prm.tiles_q = plan.tiles_q;
         prm.gq = gA;
+        if ((st = splitk_ws(dev, stream, plan, nullptr, 0, &prm.ws)) != NVFP4_OK) return st;
         const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
         const int sk = plan.splits > 1 ? 1 : 0;
         if (plan.bq == 16)
@@ -1043,7 +1297,7 @@ nvfp4_status nvfp4_gemm_bf16a(const void* A, float gA, const void* B, const void
     // by programmatic dependent launch).
     const size_t codes_bytes = (size_t)M * (K / 2), off_s = align_up(codes_bytes, 256);
     uint8_t* ws = nullptr;
-    if ((st = get_scratch(dev, stream, off_s + (size_t)M * (K / 16), &ws, /*act=*/true)) != NVFP4_OK) return st;
+    if ((st = get_scratch(dev, stream, off_s + (size_t)M * (K / 16), &ws, kScratchAct)) != NVFP4_OK) return st;
     if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((st = nvfp4_quantize_scaled(A, 1, M, K, gA, ws, ws + off_s, stream_)) != NVFP4_OK) return st;
     return nvfp4_gemm(ws, ws + off_s, B, sB, alpha, D, M, N, K, stream_);
@@ -1141,7 +1395,7 @@ extern "C" nvfp4_status nvfp4_gemm_sparse24(const void* A, const void* sA, const
     // written right before it).
     const size_t dense_bytes = (size_t)N * (size_t)(K / 2);
     uint8_t* dense = nullptr;
-    if ((st = get_scratch(dev, stream, dense_bytes, &dense, /*act=*/true)) != NVFP4_OK) return st;
+    if ((st = get_scratch(dev, stream, dense_bytes, &dense, kScratchAct)) != NVFP4_OK) return st;
     const long long items = (long long)N * (K / 16);
     const int threads = 256;
     const int blocks = (int)std::min<long long>((items + threads - 1) / threads, (long long)info->num_sms * 8);
@@ -1209,25 +1463,35 @@ nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA, const void* B, co
                                 int M, int N, int K, void* stream_) {
     nvfp4_status st = check_gemm_args(A, sA, B, sB, D, M, N, K);
     if (st != NVFP4_OK || M == 0 || N == 0) return st;
-    if (use_gemv(M, N, K)) {   // no scratch at all
-        int dev;
-        DeviceInfo* info;
-        if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
-        return gemv_gemm(info, A, sA, B, sB, alpha, D, M, N, K, 0u, static_cast<cudaStream_t>(stream_));
+    int dev;
+    DeviceInfo* info;
+    if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    // A few token rows: the CUDA-core kernel, which uses no scratch at all.
+    if (use_gemv(M, N, K)) return gemv_gemm(info, A, sA, B, sB, alpha, D, M, N, K, 0u, stream);
+    // Row-major scales that TMA can load (K % 256 == 0, 16-byte aligned): the
+    // tensor-core kernels lay them out on chip; the static scratch holds at
+    // most the split-K partials (or the plan runs without a K split).  The
+    // CTA-pair kernel, which needs its scales re-laid out first, is not used;
+    // its shapes run on the single-CTA persistent kernel.
+    const bool sfr = (K % 256 == 0) && aligned(sA, 16) && aligned(sB, 16);
+    uint8_t* scratch = nullptr;
+    if (sfr) {
+        if ((st = noalloc_scratch_address(dev, &scratch)) != NVFP4_OK) return st;
+        return sfr_gemm(dev, info, make_plan(M, N, K, info, true), A, sA, B, sB, alpha, D, M, N, K, 0u, stream,
+                        scratch, kNoAllocScratchBytes);
     }
-    // Scales of both operands, re-laid out, must fit the static scratch.
+    // Otherwise the scales of both operands are re-laid out into the static
+    // scratch, which they must fit (the split-K partials follow them there,
+    // or the plan runs without a K split).
     const size_t sfa_bytes = nvfp4_swizzled_scale_bytes(M, K);
     const size_t sfb_bytes = nvfp4_swizzled_scale_bytes(N, K);
     if (align_up(sfa_bytes, 256) + sfb_bytes > kNoAllocScratchBytes) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    int dev;
-    DeviceInfo* info;
-    st = current_device(&dev, &info);
-    if (st != NVFP4_OK) return st;
-    uint8_t* scratch = nullptr;
     if ((st = noalloc_scratch_address(dev, &scratch)) != NVFP4_OK) return st;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
-    const Plan plan = make_plan(M, N, K, info, /*sfr=*/false);
+    Plan plan = make_plan(M, N, K, info, /*sfr=*/false);
+    const size_t ws_off = align_up(align_up(sfa_bytes, 256) + sfb_bytes, 256);
+    if (ws_off + splitk_ws_bytes(plan) > kNoAllocScratchBytes) plan = make_plan(M, N, K, info, false, 1);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
     const void* sP = plan.swap ? sB : sA;
@@ -1258,6 +1522,8 @@ nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA, const void* B, co
     prm.k_tiles = plan.k_tiles;
     prm.tiles_q = plan.tiles_q;
     prm.prefetch_b = 0;
+    if ((st = splitk_ws(dev, stream, plan, scratch + ws_off, kNoAllocScratchBytes - ws_off, &prm.ws)) != NVFP4_OK)
+        return st;
     const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
     return launch_mode<false>(plan, info, maps, prm, grid, stream);
 }

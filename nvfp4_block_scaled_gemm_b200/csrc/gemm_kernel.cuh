@@ -35,13 +35,14 @@
 //
 // Split-K: the CTAs that share an output tile form one thread-block cluster
 // (blockIdx.x = cluster rank = K slice).  Rank r owns rows [r*128/S,
-// (r+1)*128/S) of the tile.  Every CTA stores each fp32 partial row straight
-// from registers into the owner's receive slots (distributed shared memory,
-// slot = the sender's rank; a region of its own, outside the ring); after one
-// cluster barrier each owner sums its S slots in rank order (deterministic),
-// applies alpha and stores BF16.  The cluster barrier that guarantees every
-// peer has started is arrived at kernel start and waited on just before the
-// first remote store.
+// (r+1)*128/S) of the tile.  Every CTA writes its fp32 partial tile from
+// registers to a global workspace (L2) with coalesced 16-byte stores; after
+// one cluster barrier (release/acquire at cluster scope, which orders the
+// global stores too) each owner reads its rows of all S partials back, sums
+// them in rank order (deterministic), applies alpha and stores BF16 with
+// 16-byte stores.  Moving the partials through L2 rather than distributed
+// shared memory is several times faster per SM (measured: a 64 KB partial
+// took 2.8 us to push into a peer's shared memory).
 //
 // BF16 activations (QBF16, swapped layout only): the producer brings the raw
 // BF16 Q tile (BQ rows x 256 values) by TMA instead of the FP4 tile and its
@@ -87,16 +88,9 @@ struct TileConfig {
     static constexpr int QRAW_OFF = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
     static constexpr int QRAW_BYTES = QBF16 ? BQ * 256 * 2 : 0;
     static constexpr int STAGE_BYTES = QRAW_OFF + QRAW_BYTES;
-    // split-K receive slots: one fp32 row of kPartLd floats per tile row, in
-    // a region of their own when that still leaves kScaleBuffers stages,
-    // otherwise in the ring (then written only after the whole cluster's
-    // main loops are done).
-    static constexpr int SLOT_NEED = kBM * (BQ + 4) * 4;
-    static constexpr bool OWN_SLOTS = SPLITK && (kSmemLimit - 2048 - SLOT_NEED) / STAGE_BYTES >= kScaleBuffers;
-    static constexpr int SLOT_BYTES = OWN_SLOTS ? SLOT_NEED : 0;
-    static constexpr int STAGES_FIT = (kSmemLimit - 2048 - SLOT_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES_FIT = (kSmemLimit - 2048) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SLOT_BYTES + 1024;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
     // TMEM columns: fp32 accumulator [0, BQ), then kScaleBuffers scale buffers
     // of (P: 4 steps x 4) + (Q: 4 steps x 4 x Q_BLOCKS) columns.
     static constexpr int SF_BASE = BQ < 32 ? 32 : BQ;
@@ -121,32 +115,25 @@ struct GemmParams {
     int tiles_q;              // tiles along Q; blockIdx.y = tq + tiles_q * tp
     int prefetch_b;           // B is constant: fetch its first tiles before waiting on the previous grid
     float gq;                 // QBF16: global scale of the BF16 activations
+    float4* ws;               // split-K partials: [tile][rank][BQ/4][128 rows] float4 (global workspace)
 };
 
 template <int BQ, bool SWAP>
 __device__ __forceinline__ void store_tile_chunk(const GemmParams& prm, const float (&v)[16], int p, int q0) {
+    static_assert(!SWAP, "the swapped layout is stored through shared memory");
     // v[c] is the fp32 result for (P row p, Q row q0 + c); alpha already applied.
+    // D[p][q]: 16 consecutive bf16 of one row -> two 16-byte stores.
     if (p >= prm.rows_p) return;
-    if (!SWAP) {
-        // D[p][q]: 16 consecutive bf16 of one row -> two 16-byte stores.
-        __nv_bfloat16* dst = prm.D + (size_t)p * prm.ldd + q0;
+    __nv_bfloat16* dst = prm.D + (size_t)p * prm.ldd + q0;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            if (q0 + 8 * h < prm.rows_q) {   // rows_q (= N) is a multiple of 8
-                uint4 w;
-                w.x = pack_bf16x2(v[8 * h + 0], v[8 * h + 1]);
-                w.y = pack_bf16x2(v[8 * h + 2], v[8 * h + 3]);
-                w.z = pack_bf16x2(v[8 * h + 4], v[8 * h + 5]);
-                w.w = pack_bf16x2(v[8 * h + 6], v[8 * h + 7]);
-                *reinterpret_cast<uint4*>(dst + 8 * h) = w;
-            }
-        }
-    } else {
-        // D[q][p]: lanes hold consecutive p, so each store instruction of the
-        // warp writes 32 consecutive bf16 of one output row.
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            if (q0 + c < prm.rows_q) prm.D[(size_t)(q0 + c) * prm.ldd + p] = __float2bfloat16_rn(v[c]);
+    for (int h = 0; h < 2; ++h) {
+        if (q0 + 8 * h < prm.rows_q) {   // rows_q (= N) is a multiple of 8
+            uint4 w;
+            w.x = pack_bf16x2(v[8 * h + 0], v[8 * h + 1]);
+            w.y = pack_bf16x2(v[8 * h + 2], v[8 * h + 3]);
+            w.z = pack_bf16x2(v[8 * h + 4], v[8 * h + 5]);
+            w.w = pack_bf16x2(v[8 * h + 6], v[8 * h + 7]);
+            *reinterpret_cast<uint4*>(dst + 8 * h) = w;
         }
     }
 }
@@ -191,47 +178,96 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
                  : "memory");
 }
 
-// Row stride (floats) of a partial row slot in shared memory; the +4 keeps
-// the 16-byte accesses of a warp (one row per lane) free of bank conflicts.
+// Split-K partial of this CTA in the workspace: float4 index (c4 * 128 + row)
+// of a [BQ/4][128] block per (tile, rank), so that the 32 lanes of a warp
+// (32 consecutive rows) store 512 contiguous bytes per instruction.
 template <int BQ>
-constexpr int kPartLd = BQ + 4;
+__device__ __forceinline__ float4* partial_block(const GemmParams& prm, int rank) {
+    return prm.ws + ((size_t)blockIdx.y * gridDim.x + rank) * (size_t)(BQ / 4) * kBM;
+}
 
 // Split-K reduction, run by the 128 epilogue threads of the owner (cluster
-// rank r) after the cluster barrier: its rows_per rows, summed over the S
-// slots [z][rows_per][kPartLd] in rank order, scaled by alpha and stored.
-template <int BQ, bool SWAP>
-__device__ __forceinline__ void reduce_owned_rows(const GemmParams& prm, uint32_t slots, int tp, int q_row0, int t) {
-    const int S = (int)gridDim.x, rank = (int)blockIdx.x;
+// rank `split`) after the cluster barrier: its rows_per rows of every rank's
+// partial, summed in rank order, scaled by alpha and stored as BF16 with
+// 16-byte stores.
+template <int BQ, bool SWAP, int S>
+__device__ __forceinline__ void reduce_from_workspace(const GemmParams& prm, int tp, int q_row0, int t) {
+    const int split = (int)blockIdx.x;
     const int rows_per = kBM / S;
-    const int row0 = rank * rows_per;
-    constexpr int C4 = BQ / 4;                     // float4 columns per row
-    const int n4 = rows_per * C4;
-    const uint32_t slot_bytes = (uint32_t)(rows_per * kPartLd<BQ>) * 4u;
-    for (int i = t; i < n4; i += 128) {
-        // swapped: consecutive threads take consecutive P rows (contiguous in D)
-        const int r = SWAP ? (i % rows_per) : (i / C4);
-        const int c4 = SWAP ? (i / rows_per) : (i % C4);
-        const uint32_t off = slots + (uint32_t)(r * kPartLd<BQ> + 4 * c4) * 4u;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int z = 0; z < S; ++z) {          // rank order
-            const uint4 v = ld_shared_v4(off + (uint32_t)z * slot_bytes);
-            acc.x += __uint_as_float(v.x);
-            acc.y += __uint_as_float(v.y);
-            acc.z += __uint_as_float(v.z);
-            acc.w += __uint_as_float(v.w);
-        }
-        const int p = tp * kBM + row0 + r;
-        const int q = q_row0 + 4 * c4;
-        if (p >= prm.rows_p) continue;
-        const float o[4] = {acc.x * prm.alpha, acc.y * prm.alpha, acc.z * prm.alpha, acc.w * prm.alpha};
-        if (!SWAP) {
-            if (q < prm.rows_q)   // rows_q (= N) is a multiple of 8
-                *reinterpret_cast<uint2*>(prm.D + (size_t)p * prm.ldd + q) =
-                    make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-        } else {
+    const int row0 = split * rows_per;
+    const int lane = t & 31;
+    if (SWAP) {
+        // Item (4 token columns c4, weight row r): lanes take consecutive r
+        // (coalesced float4 loads); 8 consecutive r in 8 consecutive lanes,
+        // whose sums lane r % 8 == i gathers for column 4 c4 + i and writes
+        // as D[q][p .. p+7].  Every lane runs every shuffle (uniform loop).
+        const int items = rows_per * (BQ / 4);
+        for (int base = 0; base < items; base += 128) {
+            const int it = base + t;
+            const bool live = it < items;
+            const int r = live ? it % rows_per : 0, c4 = live ? it / rows_per : 0;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (live) {
+                float4 v[S];   // every rank's load in flight at once, then the sums in rank order
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (q + j < prm.rows_q) prm.D[(size_t)(q + j) * prm.ldd + p] = __float2bfloat16_rn(o[j]);
+                for (int z = 0; z < S; ++z) v[z] = partial_block<BQ>(prm, z)[c4 * kBM + row0 + r];
+#pragma unroll
+                for (int z = 0; z < S; ++z) acc.x += v[z].x, acc.y += v[z].y, acc.z += v[z].z, acc.w += v[z].w;
+            }
+            const float a[4] = {acc.x * prm.alpha, acc.y * prm.alpha, acc.z * prm.alpha, acc.w * prm.alpha};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float g[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) g[j] = __shfl_sync(0xffffffffu, a[i], (lane & ~7) | j);
+                const int q = q_row0 + 4 * c4 + i, p = tp * kBM + row0 + r;
+                if (live && (r & 7) == i && rows_per >= 8 && q < prm.rows_q && p - i < prm.rows_p) {
+                    uint4 w;
+                    w.x = pack_bf16x2(g[0], g[1]);
+                    w.y = pack_bf16x2(g[2], g[3]);
+                    w.z = pack_bf16x2(g[4], g[5]);
+                    w.w = pack_bf16x2(g[6], g[7]);
+                    *reinterpret_cast<uint4*>(prm.D + (size_t)q * prm.ldd + (p - i)) = w;   // p - i: the group's first row
+                }
+            }
+            if (rows_per < 8 && live) {   // fewer than 8 owned rows: one BF16 per element
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int q = q_row0 + 4 * c4 + i, p = tp * kBM + row0 + r;
+                    if (q < prm.rows_q && p < prm.rows_p) prm.D[(size_t)q * prm.ldd + p] = __float2bfloat16_rn(a[i]);
+                }
+            }
+        }
+    } else {
+        // Item (token row r, 8 weight columns c8): two float4 per rank,
+        // one 16-byte store of D[p][q .. q+7]; lanes take consecutive r.
+        const int items = rows_per * (BQ / 8);
+        for (int it = t; it < items; it += 128) {
+            const int r = it % rows_per, c8 = it / rows_per;
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            float4 a[S], b[S];   // every rank's loads in flight at once, then the sums in rank order
+#pragma unroll
+            for (int z = 0; z < S; ++z) {
+                const float4* blk = partial_block<BQ>(prm, z);
+                a[z] = blk[(2 * c8) * kBM + row0 + r];
+                b[z] = blk[(2 * c8 + 1) * kBM + row0 + r];
+            }
+#pragma unroll
+            for (int z = 0; z < S; ++z) {
+                acc[0] += a[z].x, acc[1] += a[z].y, acc[2] += a[z].z, acc[3] += a[z].w;
+                acc[4] += b[z].x, acc[5] += b[z].y, acc[6] += b[z].z, acc[7] += b[z].w;
+            }
+            const int p = tp * kBM + row0 + r, q = q_row0 + 8 * c8;
+            if (p < prm.rows_p && q < prm.rows_q) {   // rows_q (= N) is a multiple of 8
+                uint4 w;
+                w.x = pack_bf16x2(acc[0] * prm.alpha, acc[1] * prm.alpha);
+                w.y = pack_bf16x2(acc[2] * prm.alpha, acc[3] * prm.alpha);
+                w.z = pack_bf16x2(acc[4] * prm.alpha, acc[5] * prm.alpha);
+                w.w = pack_bf16x2(acc[6] * prm.alpha, acc[7] * prm.alpha);
+                *reinterpret_cast<uint4*>(prm.D + (size_t)p * prm.ldd + q) = w;
+            }
         }
     }
 }
@@ -248,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // [ring: S stages][split-K receive slots][barriers]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES + C::SLOT_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
     // bars: [0,S) full, [S,2S) empty, [2S,2S+NB) sf_ready, [2S+NB] accum,
     //       [2S+NB+1] cvt (QBF16: the four writer warps quantized a K tile)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + NB + 2);
@@ -303,7 +339,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (SPLITK) cluster_arrive_relaxed();   // "this CTA has started" (waited on before the push)
     // Everything above overlaps the previous kernel's tail when launched with
     // programmatic stream serialisation; global memory is touched only below.
     grid_launch_dependents();
@@ -537,39 +572,74 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]) * prm.alpha;
-                store_tile_chunk<BQ, SWAP>(prm, v, p, q_row0 + c0);
+                if (!SWAP) {
+                    store_tile_chunk<BQ, false>(prm, v, p, q_row0 + c0);
+                } else {
+                    // D[q][p]: the warp's 32 rows p x 16 columns q go through
+                    // shared memory (stage 0, free once every MMA is done and
+                    // nothing else reads it) and leave as 16-byte pieces of 8
+                    // consecutive p.
+                    const uint32_t tb = smem_base + (uint32_t)(quad * 1024);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(v[c]);
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(tb + (uint32_t)(c * 64 + lane * 2)),
+                                     "h"(*reinterpret_cast<const uint16_t*>(&h))
+                                     : "memory");
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int idx = lane + 32 * h, c = idx >> 2, part = idx & 3;
+                        const int q = q_row0 + c0 + c, pp = tp * kBM + quad * 32 + part * 8;
+                        const uint4 val = ld_shared_v4(tb + (uint32_t)(c * 64 + part * 16));
+                        if (q < prm.rows_q && pp < prm.rows_p)   // rows_p (= N) is a multiple of 8
+                            *reinterpret_cast<uint4*>(prm.D + (size_t)q * prm.ldd + pp) = val;
+                    }
+                    __syncwarp();
+                }
             }
         }
     }
 
     if (SPLITK) {
-        if (C::OWN_SLOTS) {
-            cluster_wait();   // every peer has started: its receive slots may be written
-        } else {
-            cluster_wait();
-            cluster_sync();   // every peer is past its main loop: its ring may be written
-        }
-        const uint32_t slots = C::OWN_SLOTS ? smem_base + S * C::STAGE_BYTES : smem_base;
+        // Partial tile -> workspace (after the grid dependency wait, which
+        // every epilogue thread passed at the start), one cluster barrier,
+        // then each owner's sum.
         if (warp >= 2 && !*abort_flag) {
             const int quad = warp & 3;
             const int row = quad * 32 + lane;
-            const int rows_per = kBM / splits;
-            const uint32_t owner = (uint32_t)(row / rows_per);
-            const uint32_t local = slots + (uint32_t)((split * rows_per + row % rows_per) * kPartLd<BQ>) * 4u;
-            const uint32_t dst = cluster_rank_addr(local, owner);
+            float4* dst = partial_block<BQ>(prm, split);
             const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+            constexpr int CW = BQ < 32 ? 16 : 32;   // columns per TMEM load (one wait each)
 #pragma unroll 1
-            for (int c0 = 0; c0 < BQ; c0 += 16) {
-                uint32_t r[16];
-                tmem_load_16(t_quad + c0, r);
+            for (int c0 = 0; c0 < BQ; c0 += CW) {
+                uint32_t r[32];
+                if (CW == 32) {
+                    tmem_load_32(t_quad + c0, r);
+                } else {
+                    uint32_t h[16];
+                    tmem_load_16(t_quad + c0, h);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) r[c] = h[c];
+                }
                 tmem_wait_load();
 #pragma unroll
-                for (int c = 0; c < 16; c += 4)
-                    st_cluster_v4(dst + 4u * (c0 + c), r[c], r[c + 1], r[c + 2], r[c + 3]);
+                for (int c = 0; c < CW / 4; ++c)
+                    dst[(c0 / 4 + c) * kBM + row] = make_float4(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]),
+                                                                __uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3]));
             }
         }
-        cluster_sync();   // every partial row has reached its owner; no remote access after this
-        if (warp >= 2 && !*abort_flag) reduce_owned_rows<BQ, SWAP>(prm, slots, tp, q_row0, threadIdx.x - 64);
+        cluster_sync();   // every rank's partial is in the workspace and visible to the cluster
+        if (warp >= 2 && !*abort_flag) {
+            const int t = threadIdx.x - 64;
+            switch (splits) {
+                case 2: reduce_from_workspace<BQ, SWAP, 2>(prm, tp, q_row0, t); break;
+                case 4: reduce_from_workspace<BQ, SWAP, 4>(prm, tp, q_row0, t); break;
+                case 8: reduce_from_workspace<BQ, SWAP, 8>(prm, tp, q_row0, t); break;
+                default: reduce_from_workspace<BQ, SWAP, 16>(prm, tp, q_row0, t); break;
+            }
+        }
     }
 
     tc_fence_before();

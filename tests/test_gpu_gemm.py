@@ -266,20 +266,58 @@ def test_shape_mismatch_raises(nv):
 
 
 # ------------------------------------------------------------------ full-size sampled parity
-FULL = [(m, 768, 6144, "normal", 1100 + i) for i, m in enumerate(synth.ATTN_SWEEP_M)] + [
-    (2048, 2048, 6144, "moe", 1205), (512, 256, 6144, "moe", 1214), (2048, 2048, 6144, "uniform", 1300)]
+# Every configured shape at full size, on the configs' own inputs (seeded fp32
+# sources quantized by the oracle): the single 8 x 768 x 6144 GEMM, the
+# attention sweep, the MoE sweep (N = 2048 and 256) and the saturation sweep
+# ("Peeling the Kernel Onion", sections "The Chain of Reasoning", "The
+# Benchmark Design" and "The Results").  Outputs are sampled: random
+# positions plus every tile-edge row and column (boundary_samples).
+CONFIG_SHAPES = ([("single_8x768x6144", 8, 768, 6144, "normal", 1000)] + synth.attention_sweep() +
+                 synth.moe_sweep() + synth.saturation_sweep())
 
 
-@pytest.mark.parametrize("M,N,K,kind,seed", FULL)
-def test_full_size_sampled(nv, M, N, K, kind, seed):
-    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, kind, seed)
-    got = run_gemm(nv, ca, sa, cb, sb, alpha)
-    rng = np.random.default_rng(seed)
-    n = 3000
-    rows = np.concatenate([rng.integers(0, M, n), [0, M - 1, M - 1]])
-    cols = np.concatenate([rng.integers(0, N, n), [0, N - 1, 0]])
+_problems = {}
+
+
+def config_problem(M, N, K, kind, seed):
+    key = (M, N, K, kind, seed)
+    if key not in _problems:
+        _problems.clear()            # keep at most one large problem in host memory
+        _problems[key] = quantized_problem(M, N, K, kind, seed)
+    return _problems[key]
+
+
+def run_gemm_sampled(nv, ca, sa, cb, sb, alpha, rows, cols):
+    M, N = ca.shape[0], cb.shape[0]
+    assert rows.min() >= 0 and rows.max() < M and cols.min() >= 0 and cols.max() < N   # checked before any gather
+    D = nv.gemm(dev(ca), dev(sa), dev(cb), dev(sb), alpha)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    r = torch.from_numpy(rows.astype(np.int64)).cuda()
+    c = torch.from_numpy(cols.astype(np.int64)).cuda()
+    return D[r, c].float().cpu().numpy()
+
+
+# The saturation shapes run twice in a row: on the CTA-pair kernel (the
+# default) and with NVFP4_GEMM_PAIR=0 on the single-CTA persistent kernel.
+CONFIG_CASES = []
+for _c in CONFIG_SHAPES:
+    if _c[0].startswith("sat_"):
+        CONFIG_CASES += [_c + ("pair",), _c + ("single_cta",)]
+    else:
+        CONFIG_CASES.append(_c + ("default",))
+
+
+@pytest.mark.parametrize("name,M,N,K,kind,seed,kernel", CONFIG_CASES,
+                         ids=[f"{c[0]}-{c[6]}" for c in CONFIG_CASES])
+def test_config_shape_sampled(nv, monkeypatch, name, M, N, K, kind, seed, kernel):
+    if kernel == "single_cta":
+        monkeypatch.setenv("NVFP4_GEMM_PAIR", "0")
+    ca, sa, cb, sb, alpha = config_problem(M, N, K, kind, seed)
+    rows, cols = boundary_samples(M, N, seed + (kernel == "single_cta"), n_random=3000)
+    got = run_gemm_sampled(nv, ca, sa, cb, sb, alpha, rows, cols)
     _, ref, ad = oracle.gemm_sampled(ca, sa, cb, sb, alpha, M, N, K, rows, cols)
-    assert not violations(got[rows, cols], ref, ad).any()
+    assert not violations(got, ref, ad).any()
 
 
 # ------------------------------------------------------------------ bounded waits
@@ -386,11 +424,11 @@ def boundary_samples(M, N, seed, n_random=4000, edge=256):
     rng = np.random.default_rng(seed)
     rows = [rng.integers(0, M, n_random)]
     cols = [rng.integers(0, N, n_random)]
-    for r in sorted({0, 127, 128, min(255, M - 1), min(256, M - 1), M - 1}):
+    for r in sorted({x for x in (0, 127, 128, 255, 256, M - 1) if x < M}):
         c = np.arange(0, N, max(1, N // edge))
         rows.append(np.full(c.size, r))
         cols.append(c)
-    for c in sorted({0, 127, 128, min(255, N - 1), min(256, N - 1), N - 1}):
+    for c in sorted({x for x in (0, 127, 128, 255, 256, N - 1) if x < N}):
         r = np.arange(0, M, max(1, M // edge))
         rows.append(r)
         cols.append(np.full(r.size, c))

@@ -149,3 +149,45 @@ def test_grouped_more_experts_than_the_order_table(nv):
     _, ref, ad = oracle.grouped_gemm(A, sA, B, sB, alpha, off, G, Mt, N, K)
     got = run(nv, A, sA, B, sB, alpha, off)
     assert not violations(got, ref, ad).any()
+
+
+def test_grouped_full_size_recipe_sampled_experts(nv):
+    # The grouped configuration itself: 256 experts x [2048 x 6144], 512
+    # tokens top-8 with Zipf(1.1) routing, tokens N(0,1) with 1% x20 outliers
+    # (one global scale), and for the checked experts weights N(0, 0.02)
+    # quantized by the oracle with one global scale per expert (alpha[e] =
+    # gA * gB_e).  Quantizing all 256 experts on the host would take minutes,
+    # so ten experts follow the recipe -- the busiest, the least busy active
+    # ones and a random draw -- and the rest hold random codes (their rows are
+    # computed but not checked).  Every row of a checked expert is checked at
+    # sampled columns and at the first and last column.
+    G, N, K = synth.MOE_EXPERTS, synth.MOE_N, synth.HIDDEN_K
+    r = synth.moe_routing()
+    Mt = int(r.row_offsets[-1])
+    counts = np.diff(r.row_offsets)
+    X = synth.activations_with_outliers(synth.MOE_TOKENS, K, 1400)
+    ct, st_, ga = oracle.quantize(X)
+    A, sA = ct[r.token_of_row], st_[r.token_of_row]
+    rng = np.random.default_rng(1401)
+    active = np.flatnonzero(counts)
+    by_load = active[np.argsort(counts[active], kind="stable")]
+    checked = sorted(set(by_load[-3:].tolist()) | set(by_load[:3].tolist()) |
+                     set(rng.choice(active, 4, replace=False).tolist()))
+    B = synth.random_codes(G * N, K, 1402).reshape(G, N, K // 2)
+    sB = synth.random_scales(G * N, K, 1403, lo=0x28, hi=0x38).reshape(G, N, K // 16)
+    alpha = np.full(G, 1.0e-3, np.float32)
+    for e in checked:
+        cb, sb, gb = oracle.quantize(synth.normal(N, K, 1500 + e, std=0.02))
+        B[e], sB[e] = cb, sb
+        alpha[e] = np.float32(ga) * np.float32(gb)
+    D = nv.grouped_gemm(dev(A), dev(sA), dev(B), dev(sB), dev(alpha), dev(r.row_offsets.astype(np.int32)))
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    for e in checked:
+        r0, r1 = int(r.row_offsets[e]), int(r.row_offsets[e + 1])
+        rows = np.repeat(np.arange(r0, r1), 34)
+        cols = np.concatenate([np.concatenate([[0, N - 1], rng.integers(0, N, 32)]) for _ in range(r1 - r0)])
+        assert rows.min() >= 0 and rows.max() < Mt and cols.min() >= 0 and cols.max() < N   # before the gather
+        got = D[torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()].float().cpu().numpy()
+        _, ref, ad = oracle.gemm_sampled(A, sA, B[e], sB[e], float(alpha[e]), Mt, N, K, rows, cols)
+        assert not violations(got, ref, ad).any(), f"expert {e}"
