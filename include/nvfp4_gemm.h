@@ -317,6 +317,31 @@ nvfp4_status nvfp4_gemm_sparse24(const void* A, const void* sA,
                                  float alpha, void* D,
                                  int M, int N, int K, unsigned flags, void* stream);
 
+/*
+ * nvfp4_gemm_mxfp4 -- D = alpha * A * B^T with MXFP4 operands, the OCP
+ * microscaling format the same tensor-core instruction family takes
+ * (tcgen05.mma kind::mxf4, block32): E2M1 codes packed as for nvfp4_gemm,
+ * with one E8M0 scale per 32 values along K (byte e = 2^(e - 127); 255 is
+ * NaN and must not occur).  The pages use NVFP4 only; this is the format's
+ * sibling, exact up to the fp32 accumulation like nvfp4_gemm.
+ *   A  [M][K/2], sA [M][K/32] (E8M0 bytes), B [N][K/2], sB [N][K/32];
+ *   alpha fp32 (no global scales in this format; kept for the same call
+ *   shape); D bf16 [M][N]; flags as for nvfp4_gemm_ex.
+ *   Requirements: K % 64 == 0, N % 8 == 0; A, B, D 16-byte aligned (scales
+ *   any alignment).  M == 0 or N == 0 is a no-op.
+ *   Up to 4 token rows run on the CUDA cores (exact block sums, each scaled
+ *   by 2^(ea + eb - 254) with ldexpf, fp32 sum); above that both operands'
+ *   scales are re-laid out into per-stream scratch (may cudaMalloc on a
+ *   stream's first use of a size) and the tensor-core kernel runs.  The
+ *   partial sums are fp32, so products whose scales leave the fp32 range
+ *   (about 2^-149 .. 2^127) under- or overflow.
+ *   Errors: as for nvfp4_gemm.
+ */
+nvfp4_status nvfp4_gemm_mxfp4(const void* A, const void* sA,
+                              const void* B, const void* sB,
+                              float alpha, void* D,
+                              int M, int N, int K, unsigned flags, void* stream);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int nvfp4_version(void);
 

@@ -33,7 +33,7 @@ EXPORTS = (
     "nvfp4_swizzled_scale_bytes", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_debug_wait_timeout", "nvfp4_version", "nvfp4_kernel_launches",
     "nvfp4_gemm_noalloc", "nvfp4_fp4_peak_probe", "nvfp4_quantize_scaled", "nvfp4_gemm_bf16a",
-    "nvfp4_gemm_sparse24",
+    "nvfp4_gemm_sparse24", "nvfp4_gemm_mxfp4",
 )
 
 
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_gemm_bf16a.restype = i32
         L.nvfp4_gemm_sparse24.argtypes = [P, P, P, P, P, f32, P, i32, i32, i32, ctypes.c_uint, P]
         L.nvfp4_gemm_sparse24.restype = i32
+        L.nvfp4_gemm_mxfp4.argtypes = [P, P, P, P, f32, P, i32, i32, i32, ctypes.c_uint, P]
+        L.nvfp4_gemm_mxfp4.restype = i32
         _lib = L
     return _lib
 
@@ -196,6 +198,29 @@ def gemm_sparse24(A: torch.Tensor, sA: torch.Tensor, Bv: torch.Tensor, Bm: torch
     _check(lib().nvfp4_gemm_sparse24(A.data_ptr(), sA.data_ptr(), Bv.data_ptr(), Bm.data_ptr(), sB.data_ptr(),
                                      float(alpha), out.data_ptr(), M, N, K, B_CONSTANT if b_constant else 0,
                                      _stream(stream)), "nvfp4_gemm_sparse24")
+    return out
+
+
+def gemm_mxfp4(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor, alpha: float,
+               out: torch.Tensor | None = None, stream=None, b_constant: bool = False) -> torch.Tensor:
+    """D[M,N] (bf16) = alpha * (A * sA) @ (B * sB)^T in MXFP4: uint8 codes
+    A [M, K/2], B [N, K/2] as for gemm(), E8M0 scales sA [M, K/32],
+    sB [N, K/32] (one per 32 values, 2^(byte - 127))."""
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D packed E2M1 tensors [rows, K/2]")
+    M, N, K = A.shape[0], B.shape[0], packed_k(A)
+    if packed_k(B) != K:
+        raise ValueError(f"K mismatch: A holds K={K}, B holds K={packed_k(B)}")
+    _need(A, "A", torch.uint8, (M, K // 2))
+    _need(B, "B", torch.uint8, (N, K // 2))
+    _need(sA, "sA", torch.uint8, (M, K // 32))
+    _need(sB, "sB", torch.uint8, (N, K // 32))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _need(out, "out", torch.bfloat16, (M, N))
+    _check(lib().nvfp4_gemm_mxfp4(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(), float(alpha),
+                                  out.data_ptr(), M, N, K, B_CONSTANT if b_constant else 0, _stream(stream)),
+           "nvfp4_gemm_mxfp4")
     return out
 
 

@@ -41,6 +41,7 @@ struct DeviceInfo {
     bool supported = false;
     int num_sms = 0;
     uint64_t smem_attr_set = 0;  // bit per kernel instantiation
+    uint64_t smem_attr_set_mx = 0;  // the same for the MXFP4 instantiations
     int pair_clusters = -1;      // co-resident 2-CTA clusters of the pair kernel (-1: not queried)
     std::map<uint32_t, int> split_clusters;   // co-resident split-K clusters per (kernel, cluster size)
 };
@@ -368,20 +369,21 @@ struct Maps {
     CUtensorMap p, q, sp, sq;
 };
 
-template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false>
+template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false, bool MX = false>
 nvfp4_status launch_gemm_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, const GemmParams& prm, dim3 grid,
                                 cudaStream_t stream) {
     using C = TileConfig<BQ, SPLITK, QBF16>;
-    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK, SFR, QBF16>;
+    auto kern = nvfp4::nvfp4_gemm_kernel<BQ, SWAP, SPLITK, SFR, QBF16, MX>;
+    uint64_t& attr_set = MX ? info->smem_attr_set_mx : info->smem_attr_set;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!(info->smem_attr_set & bit)) {
+        if (!(attr_set & bit)) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
                 return NVFP4_ERR_CUDA;
             // clusters of 16 split-K CTAs are opt-in (beyond the portable 8)
             if (SPLITK && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
                 return NVFP4_ERR_CUDA;
-            info->smem_attr_set |= bit;
+            attr_set |= bit;
         }
     }
     cudaLaunchConfig_t cfg = {};
@@ -970,6 +972,66 @@ nvfp4_status sfr_gemm(int dev, DeviceInfo* info, Plan plan, const void* A, const
     return launch_mode<true>(plan, info, maps, prm, grid, stream);
 }
 
+// The MXFP4 instantiations (scale atoms pre-laid out, never row-major tiles).
+template <bool SWAP, bool SPLITK>
+nvfp4_status launch_mx_by_bq(int bq, DeviceInfo* info, const Maps& m, const GemmParams& prm, dim3 grid,
+                             cudaStream_t stream) {
+    const int base = (SWAP ? 1 : 0) * 10 + (SPLITK ? 5 : 0);
+    switch (bq) {
+        case 16: return launch_gemm_kernel<16, SWAP, SPLITK, false, false, true>(info, 1ull << (base + 0), m, prm, grid, stream);
+        case 32: return launch_gemm_kernel<32, SWAP, SPLITK, false, false, true>(info, 1ull << (base + 1), m, prm, grid, stream);
+        case 64: return launch_gemm_kernel<64, SWAP, SPLITK, false, false, true>(info, 1ull << (base + 2), m, prm, grid, stream);
+        case 128: return launch_gemm_kernel<128, SWAP, SPLITK, false, false, true>(info, 1ull << (base + 3), m, prm, grid, stream);
+        case 256: return launch_gemm_kernel<256, SWAP, SPLITK, false, false, true>(info, 1ull << (base + 4), m, prm, grid, stream);
+        default: return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    }
+}
+
+nvfp4_status launch_swizzle_mx(const void* s, int rows, int K, void* out, cudaStream_t stream) {
+    const int pairs = (K / 64 + 1) / 2;
+    const long long lines = (long long)((rows + 127) / 128) * pairs * 32;
+    if (lines == 0) return NVFP4_OK;
+    const int threads = 256;
+    const long long blocks = (lines + threads - 1) / threads;
+    nvfp4::swizzle_scales_mx_kernel<<<(unsigned)blocks, threads, 0, stream>>>(static_cast<const uint8_t*>(s), rows,
+                                                                            K / 32, pairs, lines,
+                                                                            static_cast<uint8_t*>(out));
+    g_launches++;
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+size_t mx_atom_bytes(int rows, int K) { return (size_t)((rows + 127) / 128) * (size_t)((K / 64 + 1) / 2) * 512u; }
+
+template <int MT, int RW>
+nvfp4_status launch_gemv_mx_kernel(DeviceInfo* info, const nvfp4::GemvMxParams& prm, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemv_mx_kernel<MT, RW>;
+    static const int per_sm = [kern] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, nvfp4::kGemvThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            b = 0;
+        }
+        return b > 0 ? b : 1;
+    }();
+    const int groups = (prm.N + RW - 1) / RW;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(groups, per_sm * info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGemvThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
 nvfp4_status check_gemm_args(const void* A, const void* sA, const void* B, const void* sB, const void* D, int M,
                              int N, int K) {
     if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
@@ -1529,3 +1591,79 @@ nvfp4_status nvfp4_gemm_noalloc(const void* A, const void* sA, const void* B, co
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// MXFP4 GEMM (nvfp4_gemm_mxfp4).
+// ---------------------------------------------------------------------------
+extern "C" nvfp4_status nvfp4_gemm_mxfp4(const void* A, const void* sA, const void* B, const void* sB, float alpha,
+                                         void* D, int M, int N, int K, unsigned flags, void* stream_) {
+    if (flags & ~NVFP4_GEMM_B_CONSTANT) return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!A || !sA || !B || !sB || !D) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16)) return NVFP4_ERR_INVALID_ARG;
+    int dev;
+    DeviceInfo* info;
+    nvfp4_status st = current_device(&dev, &info);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    // One to four token rows: the CUDA-core kernel (NVFP4_GEMM_GEMV sets the
+    // row limit here too, 0 turning it off).
+    int gemv_rows = 4;
+    if (const char* e = std::getenv("NVFP4_GEMM_GEMV")) gemv_rows = std::min(4, std::max(0, std::atoi(e)));
+    if (M <= gemv_rows) {
+        nvfp4::GemvMxParams prm{};
+        prm.A = static_cast<const uint8_t*>(A);
+        prm.sA = static_cast<const uint8_t*>(sA);
+        prm.B = static_cast<const uint8_t*>(B);
+        prm.sB = static_cast<const uint8_t*>(sB);
+        prm.D = static_cast<__nv_bfloat16*>(D);
+        prm.alpha = alpha;
+        prm.M = M;
+        prm.N = N;
+        prm.K = K;
+        prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+        const int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
+        if (M == 1) return rw == 4 ? launch_gemv_mx_kernel<1, 4>(info, prm, stream) : launch_gemv_mx_kernel<1, 1>(info, prm, stream);
+        if (M == 2) return launch_gemv_mx_kernel<2, 2>(info, prm, stream);
+        return launch_gemv_mx_kernel<4, 2>(info, prm, stream);
+    }
+    // The tensor cores: both operands' scales re-laid out into atoms in
+    // per-stream scratch, then the tiled kernel's kind::mxf4 form.
+    const Plan plan = make_plan(M, N, K, info, /*sfr=*/false);
+    const void* P = plan.swap ? B : A;
+    const void* Q = plan.swap ? A : B;
+    const void* sP = plan.swap ? sB : sA;
+    const void* sQ = plan.swap ? sA : sB;
+    const int rows_p = plan.swap ? N : M;
+    const int rows_q = plan.swap ? M : N;
+    const size_t off_sfq = align_up(mx_atom_bytes(rows_p, K), 256);
+    uint8_t* ws = nullptr;
+    if ((st = get_scratch(dev, stream, off_sfq + mx_atom_bytes(rows_q, K), &ws)) != NVFP4_OK) return st;
+    Maps maps;
+    if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq))
+        return NVFP4_ERR_CUDA;
+    if ((st = launch_swizzle_mx(sP, rows_p, K, ws, stream)) != NVFP4_OK) return st;
+    if ((st = launch_swizzle_mx(sQ, rows_q, K, ws + off_sfq, stream)) != NVFP4_OK) return st;
+    maps.sp = maps.p;
+    maps.sq = maps.q;
+    GemmParams prm{};
+    prm.sfp = ws;
+    prm.sfq = ws + off_sfq;
+    prm.D = static_cast<__nv_bfloat16*>(D);
+    prm.alpha = alpha;
+    prm.rows_p = rows_p;
+    prm.rows_q = rows_q;
+    prm.K = K;
+    prm.ldd = N;
+    prm.k_tiles = plan.k_tiles;
+    prm.tiles_q = plan.tiles_q;
+    if ((st = splitk_ws(dev, stream, plan, nullptr, 0, &prm.ws)) != NVFP4_OK) return st;
+    const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
+    if (plan.swap)
+        return plan.splits > 1 ? launch_mx_by_bq<true, true>(plan.bq, info, maps, prm, grid, stream)
+                               : launch_mx_by_bq<true, false>(plan.bq, info, maps, prm, grid, stream);
+    return plan.splits > 1 ? launch_mx_by_bq<false, true>(plan.bq, info, maps, prm, grid, stream)
+                           : launch_mx_by_bq<false, false>(plan.bq, info, maps, prm, grid, stream);
+}

@@ -31,6 +31,38 @@ __global__ void swizzle_scales_kernel(const uint8_t* __restrict__ s, int rows, i
     *reinterpret_cast<uint4*>(out + (rb * steps + ks) * 512 + 16 * L) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// MXFP4 scales (E8M0, one per 32 values), row-major [rows][K/32], into the
+// 512-byte atoms the kind::mxf4 MMA reads through TMEM: atom w of a 128-row
+// block holds K steps 2w and 2w+1 (64 values each); line L is the four bytes
+// of rows L, L+32, L+64, L+96, each byte quadruple being that row's scales of
+// blocks 4w .. 4w+3 (the even step's two blocks in bytes 0-1, the odd step's
+// in bytes 2-3).  Bytes past K or past the rows are zero.  One thread per
+// line; byte loads, so any row stride works.
+__global__ void swizzle_scales_mx_kernel(const uint8_t* __restrict__ s, int rows, int kb_row, int pairs,
+                                         long long lines, uint8_t* __restrict__ out) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= lines) return;
+    const int L = (int)(idx & 31);
+    const long long t = idx >> 5;
+    const int w = (int)(t % pairs);
+    const long long rb = t / pairs;
+    uint32_t v[4];
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+        const long long r = rb * 128 + L + 32 * r1;
+        uint32_t word = 0u;
+        if (r < rows) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int kb = 4 * w + b;
+                if (kb < kb_row) word |= (uint32_t)__ldg(s + r * kb_row + kb) << (8 * b);
+            }
+        }
+        v[r1] = word;
+    }
+    *reinterpret_cast<uint4*>(out + (rb * pairs + w) * 512 + 16 * L) = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
 // The same layout for two scale tensors in one launch, K a multiple of 256:
 // one 128-thread CTA per (tensor, 128-row block, 256-element K tile).  Thread
 // t reads the 16 scale bytes of row t of the block (one request per row), the

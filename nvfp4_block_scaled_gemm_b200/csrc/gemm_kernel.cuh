@@ -272,12 +272,17 @@ __device__ __forceinline__ void reduce_from_workspace(const GemmParams& prm, int
     }
 }
 
-template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false>
+// MX: the MXFP4 form (E8M0 scale per 32 values, kind::mxf4 block32), with
+// scales pre-laid out in 512-byte atoms of two K steps each (non-SFR only):
+// the atoms of a K tile are two per 128-row block instead of four, and step j
+// reads TMEM scale word j / 2 at byte 2 * (j % 2).
+template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false, bool MX = false>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                       const GemmParams prm) {
     static_assert(!QBF16 || (SWAP && SFR && BQ <= 64), "BF16 activations: swapped layout, row-major scale tiles");
+    static_assert(!MX || (!SFR && !QBF16), "MXFP4: pre-laid-out scale atoms");
     using C = TileConfig<BQ, SPLITK, QBF16>;
     constexpr int S = C::STAGES;
     constexpr int NB = kScaleBuffers;
@@ -409,16 +414,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
                     load_q(st, full_bar(s), kt);
                 } else {
+                    // atoms per 128-row block: one per K step (NVFP4) or per
+                    // pair of K steps (MXFP4)
                     const int steps = min(4, steps_total - 4 * kt);
-                    const uint32_t sf_bytes = (uint32_t)steps * kAtomBytes;
+                    const int atoms_total = MX ? (steps_total + 1) / 2 : steps_total;
+                    const int atom0 = MX ? 2 * kt : 4 * kt;
+                    const uint32_t sf_bytes = (uint32_t)(MX ? (steps + 1) / 2 : steps) * kAtomBytes;
                     mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + C::Q_BYTES + sf_bytes * (1 + q_blocks));
                     tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
                     tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(s), kt * kStageKBytes, q_row0, pol_q);
                     bulk_load(st + C::P_BYTES + C::Q_BYTES,
-                              prm.sfp + ((size_t)tp * steps_total + 4 * kt) * kAtomBytes, sf_bytes, full_bar(s));
+                              prm.sfp + ((size_t)tp * atoms_total + atom0) * kAtomBytes, sf_bytes, full_bar(s));
                     for (int b = 0; b < q_blocks; ++b) {
                         bulk_load(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + b * 4 * kAtomBytes,
-                                  prm.sfq + ((size_t)(q_block0 + b) * steps_total + 4 * kt) * kAtomBytes, sf_bytes,
+                                  prm.sfq + ((size_t)(q_block0 + b) * atoms_total + atom0) * kAtomBytes, sf_bytes,
                                   full_bar(s));
                     }
                 }
@@ -439,8 +448,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t st = smem_base + s * C::STAGE_BYTES;
                 const uint32_t sf = tmem + C::SF_BASE + b * C::SF_STRIDE;
                 for (int j = 0; j < steps; ++j) {
-                    tc_mma_nvf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
-                                idesc, sf + 4 * j, sf + 16 + 4 * C::Q_BLOCKS * j, (it > 0 || j > 0) ? 1u : 0u);
+                    if (MX) {
+                        // the atoms' word (j / 2) landed in TMEM column group j / 2
+                        tc_mma_mxf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
+                                    (j & 1) ? idesc_mxf4(kBM, BQ, 2) : idesc_mxf4(kBM, BQ, 0), sf + 4 * (j >> 1),
+                                    sf + 16 + 4 * C::Q_BLOCKS * (j >> 1), (it > 0 || j > 0) ? 1u : 0u);
+                    } else {
+                        tc_mma_nvf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::P_BYTES + 32 * j),
+                                    idesc, sf + 4 * j, sf + 16 + 4 * C::Q_BLOCKS * j, (it > 0 || j > 0) ? 1u : 0u);
+                    }
                 }
                 // one commit frees both the ring stage and the TMEM scale
                 // buffer this K tile used

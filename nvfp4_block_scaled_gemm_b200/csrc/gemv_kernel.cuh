@@ -311,4 +311,124 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_kernel(const GemvPara
     }
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4 (OCP microscaling: E2M1 values, one E8M0 scale 2^(byte - 127) per 32
+// values) for a handful of token rows, on the CUDA cores.  A 16-byte chunk of
+// codes is exactly one scale block, so each thread reads one scale byte per
+// chunk and operand.  The chunk's 32 products are summed exactly as in the
+// NVFP4 kernel (two f16x2 chains of 16 values, each exact, added in fp32),
+// then scaled by 2^(ea + eb - 254) with ldexpf (exact while the result is an
+// fp32 number) and added to the fp32 sum over chunks; the CTA's sums meet in
+// a fixed order.  No prefetch across row groups: the decode shapes have one
+// or two groups per CTA.
+struct GemvMxParams {
+    const uint8_t* A;    // [M][K/2] E2M1 codes
+    const uint8_t* sA;   // [M][K/32] E8M0 scales
+    const uint8_t* B;    // [N][K/2]
+    const uint8_t* sB;   // [N][K/32]
+    __nv_bfloat16* D;    // [M][N]
+    float alpha;
+    int M, N, K;
+    int prefetch_b;      // B is constant: load its first chunks before waiting on the previous grid
+};
+
+__device__ __forceinline__ uint32_t ld_stream_u8(const void* p) {
+    unsigned short v;
+    asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+template <int MT, int RW>
+__global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_mx_kernel(const GemvMxParams prm) {
+    constexpr int NV = RW * MT;
+    __shared__ float red[2][kGemvWarps][NV];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int kc = prm.K >> 5;                        // 16-byte chunks (= scale blocks) per row
+    const size_t row_bytes = (size_t)prm.K >> 1;
+    const size_t srow_bytes = (size_t)prm.K >> 5;
+    const int M = prm.M;
+    const int group_stride = gridDim.x * RW;
+
+    uint4 bq[kGemvGroup][RW];
+    uint32_t bs[kGemvGroup][RW];
+    auto load_group = [&](int n0, int c0) {
+#pragma unroll
+        for (int g = 0; g < kGemvGroup; ++g) {
+            const int c = c0 + g * kGemvThreads;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const int n = min(n0 + r, prm.N - 1);
+                if (c < kc) {
+                    bq[g][r] = ld_stream_v4(prm.B + (size_t)n * row_bytes + 16 * (size_t)c);
+                    bs[g][r] = ld_stream_u8(prm.sB + (size_t)n * srow_bytes + (size_t)c);
+                } else {
+                    bq[g][r] = make_uint4(0u, 0u, 0u, 0u);
+                    bs[g][r] = 127u;
+                }
+            }
+        }
+    };
+
+    grid_launch_dependents();
+    const int step = kGemvGroup * kGemvThreads;
+    int n0 = blockIdx.x * RW;
+    if (prm.prefetch_b && n0 < prm.N) load_group(n0, t);   // only B is touched before the wait
+    grid_dependency_wait();
+
+    for (int it = 0; n0 < prm.N; n0 += group_stride, ++it) {
+        float acc[RW][MT];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+        for (int c0 = t; c0 < kc; c0 += step) {
+            if (!(it == 0 && c0 == t && prm.prefetch_b)) load_group(n0, c0);
+#pragma unroll
+            for (int g = 0; g < kGemvGroup; ++g) {
+                const int c = c0 + g * kGemvThreads;
+                if (c >= kc) break;
+                uint32_t bh[RW][16];
+#pragma unroll
+                for (int r = 0; r < RW; ++r) decode_chunk(bq[g][r], bh[r]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m < M) {
+                        const uint4 aq = ld_cached_v4(prm.A + (size_t)m * row_bytes + 16 * (size_t)c);
+                        const int ea = (int)__ldg(prm.sA + (size_t)m * srow_bytes + (size_t)c);
+                        uint32_t ah[16];
+                        decode_chunk(aq, ah);
+#pragma unroll
+                        for (int r = 0; r < RW; ++r) {
+                            const float blk = block_dot(ah, bh[r]) + block_dot(ah + 8, bh[r] + 8);   // exact
+                            acc[r][m] += ldexpf(blk, ea + (int)bs[g][r] - 254);
+                        }
+                    }
+                }
+            }
+        }
+
+        float v[NV];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) v[r * MT + m] = acc[r][m];
+        warp_reduce_scatter<NV>(v, lane);
+        float (*rb)[NV] = red[it & 1];
+        if (gemv_writer_lane<NV>(lane)) {
+#pragma unroll
+            for (int j = 0; j < (NV >= 32 ? NV / 32 : 1); ++j) rb[warp][gemv_reduced_index<NV>(lane, j)] = v[j];
+        }
+        __syncthreads();
+        for (int i = t; i < NV; i += kGemvThreads) {
+            const int r = i / MT, m = i % MT;
+            if (m < M && n0 + r < prm.N) {
+                float sum = rb[0][i];
+#pragma unroll
+                for (int w = 1; w < kGemvWarps; ++w) sum += rb[w][i];
+                prm.D[(size_t)m * prm.N + n0 + r] = __float2bfloat16_rn(sum * prm.alpha);
+            }
+        }
+    }
+}
+
 }  // namespace nvfp4

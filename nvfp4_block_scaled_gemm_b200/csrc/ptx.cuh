@@ -287,6 +287,21 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// D(tmem) (+)= (A * sfA) x (B * sfB)^T for one K=64 step of E2M1 operands with
+// UE8M0 scales, one scale per 32 elements (the OCP MX format): each 32-bit
+// TMEM scale word holds two K steps' pairs of scales, the instruction
+// descriptor's scale-factor IDs pick the half.
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // Each thread of the warp reads 16 consecutive 32-bit columns of its TMEM lane.
 __device__ __forceinline__ void tmem_load_16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -372,6 +387,15 @@ __device__ __forceinline__ uint64_t desc_scale_atom(uint32_t saddr) {
 // (M >> 4), N in bits 17-22 (N >> 3).
 __host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// Instruction descriptor of kind::mxf4: A and B E2M1 (format code 1), both
+// K-major, UE8M0 scales (bit 23), M in bits 24-28 (M >> 4), N in bits 17-22
+// (N >> 3), and the scale-factor IDs of A (bits 29-30) and B (bits 4-5): the
+// byte of the 32-bit TMEM scale word where this step's scales start (0 or 2).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n, int sf_id) {
+    return ((uint32_t)sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(m >> 4) << 24) | ((uint32_t)sf_id << 29);
 }
 
 // ------------------------------------------------- programmatic dependent launch
