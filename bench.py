@@ -729,7 +729,7 @@ def run_chain(args, layers=8):
                     nv.gemm_bf16a(a, g_act[li], cb, sb, g_act[li] * gb, out=bufs[li], stream=stream)
                 else:
                     cq, sq = nv.quantize_scaled(a, g_act[li], stream=stream)
-                    nv.gemm(cq, sq, cb, sb, g_act[li] * gb, out=bufs[li], stream=stream)
+                    nv.gemm(cq, sq, cb, sb, g_act[li] * gb, out=bufs[li], stream=stream, b_constant=True)
                 a = bufs[li]
 
         def time_chain(fused):
@@ -799,7 +799,8 @@ def run_decode(args):
                     for k in keys:
                         os.environ.pop(k, None)
                     os.environ.update(env)
-                    us = time_single_shape(nv, torch, dev, M, Nn, Kk, "moe", 1700 + M, min(args.steps, 2000), stream)
+                    us = time_single_shape(nv, torch, dev, M, Nn, Kk, "moe", 1700 + M, min(args.steps, 2000), stream,
+                                           b_constant=True)
                     row[name] = round(us, 2)
                 row["default_hbm_frac"] = round(accounting.gemm_bytes(M, Nn, Kk) / row["default"] / 1e3 / hbm_gbs, 4)
                 rows.append(row)
@@ -810,7 +811,8 @@ def run_decode(args):
             else:
                 os.environ[k] = v
     return {"workload": "decode: M in {1,2,4,8} on the attention, MoE and two larger weight shapes, tensor-core vs "
-                        "CUDA-core kernel (us per GEMM, graph-replayed back-to-back calls, rotating buffers > L2)",
+                        "CUDA-core kernel (us per GEMM, graph-replayed back-to-back calls, rotating buffers > L2, "
+                        "constant weights)",
             "hbm_gbs": hbm_gbs, "shapes": rows}
 
 
@@ -876,8 +878,9 @@ def run_sparse(args):
                 assert nv.get_device_error(stream) == 0
                 return e0.elapsed_time(e1) * 1e3 / (reps * R)
 
-            us_dense = timed(lambda: [nv.gemm(ca, sa, b, s, alpha, out=o, stream=stream) for (b, s, o) in dense_sets])
-            us_sparse = timed(lambda: [nv.gemm_sparse24(ca, sa, v, m, s, alpha, out=o, stream=stream)
+            us_dense = timed(lambda: [nv.gemm(ca, sa, b, s, alpha, out=o, stream=stream, b_constant=True)
+                                      for (b, s, o) in dense_sets])
+            us_sparse = timed(lambda: [nv.gemm_sparse24(ca, sa, v, m, s, alpha, out=o, stream=stream, b_constant=True)
                                        for (v, m, s, o) in sparse_sets])
             sparse_bytes = M * Kk // 2 + M * Kk // 16 + Nn * Kk // 4 + 2 * Nn * Kk // 16 + 2 * M * Nn
             rows.append({"M": M, "N": Nn, "K": Kk, "us_dense": round(us_dense, 2), "us_sparse": round(us_sparse, 2),
@@ -885,6 +888,65 @@ def run_sparse(args):
                          "sparse_hbm_frac": round(sparse_bytes / us_sparse / 1e3 / hbm_gbs, 4)})
     return {"workload": "2:4-sparse weights vs dense on decode shapes (us per GEMM, graph-replayed back-to-back "
                         "calls, rotating buffers > 4x L2)", "hbm_gbs": hbm_gbs, "shapes": rows}
+
+
+def run_mxfp4(args):
+    """MXFP4 (nvfp4_gemm_mxfp4) on the attention and MoE shapes, graph-replayed
+    back-to-back calls over rotating buffers (> 4x L2), us per GEMM, beside
+    the NVFP4 GEMM of the same shape.  Inputs are random codes and E8M0
+    scales near 1 (the GEMM's work does not depend on the values)."""
+    import torch
+    import nvfp4_block_scaled_gemm_b200 as nv
+    dev = torch.device("cuda", 0)
+    nv.lib()
+    hbm_gbs = load_peaks()[0]
+    stream = torch.cuda.Stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    rows = []
+    for (M, Nn, Kk) in ((1, 768, 6144), (16, 768, 6144), (128, 768, 6144), (512, 768, 6144), (1, 2048, 6144),
+                        (64, 2048, 6144), (2048, 2048, 6144)):
+        g = torch.Generator(device=dev)
+        g.manual_seed(M + Nn)
+        a = torch.randint(0, 256, (M, Kk // 2), generator=g, device=dev, dtype=torch.uint8)
+        b = torch.randint(0, 256, (Nn, Kk // 2), generator=g, device=dev, dtype=torch.uint8)
+        sa = torch.randint(120, 134, (M, Kk // 32), generator=g, device=dev, dtype=torch.uint8)
+        sb = torch.randint(120, 134, (Nn, Kk // 32), generator=g, device=dev, dtype=torch.uint8)
+        nbytes = M * Kk // 2 + Nn * Kk // 2 + (M + Nn) * Kk // 32 + 2 * M * Nn
+        R = int(max(2, min(64, -(-4 * l2 // nbytes))))
+        sets = [(a.clone(), sa.clone(), b.clone(), sb.clone(), torch.empty((M, Nn), dtype=torch.bfloat16, device=dev))
+                for _ in range(R)]
+
+        def enqueue():
+            for x in sets:
+                nv.gemm_mxfp4(x[0], x[1], x[2], x[3], 1.0, out=x[4], stream=stream, b_constant=True)
+
+        with torch.cuda.stream(stream):
+            enqueue()
+        stream.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            enqueue()
+        reps = max(1, min(args.steps, 2000) // R)
+        with torch.cuda.stream(stream):
+            gr.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                gr.replay()
+            e1.record(stream)
+        stream.synchronize()
+        assert nv.get_device_error(stream) == 0
+        us = e0.elapsed_time(e1) * 1e3 / (reps * R)
+        us_nv = time_single_shape(nv, torch, dev, M, Nn, Kk, "normal", 1600 + M, min(args.steps, 2000), stream,
+                                  b_constant=True)
+        rows.append({"M": M, "N": Nn, "K": Kk, "us_mxfp4": round(us, 2), "us_nvfp4": round(us_nv, 2),
+                     "mxfp4_GBps": round(nbytes / us / 1e3, 1), "mxfp4_hbm_frac": round(nbytes / us / 1e3 / hbm_gbs, 4),
+                     "mxfp4_TFLOPS": round(2 * M * Nn * Kk / us / 1e6, 1)})
+    return {"workload": "MXFP4 GEMM (E8M0 scale per 32 values) vs NVFP4 on the same shapes, us per GEMM "
+                        "(graph-replayed back-to-back calls, rotating buffers > 4x L2, constant weights)",
+            "hbm_gbs": hbm_gbs, "shapes": rows}
 
 
 def main():
@@ -898,7 +960,7 @@ def main():
     ap.add_argument("--no-b-constant", action="store_true",
                     help="call the GEMMs without NVFP4_GEMM_B_CONSTANT (the weights are constant either way)")
     ap.add_argument("--workload", choices=["attn", "moe", "saturation", "grouped", "chain", "pages", "decode",
-                                           "sparse"],
+                                           "sparse", "mxfp4"],
                     default="attn",
                     help="attn (default) prints the benchmark line; the others print a per-shape report")
     args = ap.parse_args()
@@ -923,6 +985,8 @@ def main():
                 print(json.dumps(run_decode(args)), flush=True)
             elif args.workload == "sparse":
                 print(json.dumps(run_sparse(args)), flush=True)
+            elif args.workload == "mxfp4":
+                print(json.dumps(run_mxfp4(args)), flush=True)
             else:
                 shapes = {"moe": synth.moe_sweep, "pages": synth.pages_sweep}.get(args.workload, synth.saturation_sweep)()
                 print(json.dumps(run_shapes(args, shapes, args.workload)), flush=True)
