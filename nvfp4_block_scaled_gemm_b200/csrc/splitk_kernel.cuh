@@ -211,10 +211,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
             if (lane == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
             return __shfl_sync(0xffffffffu, ok, 0) != 0;
         };
-        // Row-major scale tile (128 rows x 16 bytes) at `base` -> four atoms
-        // in place, visible to the tensor core's copies; then lane 0 copies
-        // them to TMEM columns col + 4j.
-        auto atoms_to_tmem = [&](uint32_t base, uint32_t col) {
+        auto sf_col = [&](int s) { return tmem + (uint32_t)(C::ACC_COLS + s * C::SF_STRIDE); };
+        // Row-major scale tile at `base` -> four atoms in place (the warp's
+        // loads first, then its stores), not yet fenced for the tensor core.
+        auto build_atoms = [&](uint32_t base) {
             uint32_t w[16];
             gather_scale_words<true>(base, lane, w);   // w[4j + r1] = step j of row lane + 32 r1
             __syncwarp();
@@ -223,15 +223,25 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + 512u * j + 16u * lane),
                              "r"(w[4 * j]), "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
                              : "memory");
+        };
+        auto copy_atoms = [&](uint32_t base, uint32_t col) {   // lane 0, after the fence
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tc_copy_32x128b_x4(col + 4 * j, desc_scale_atom(base + 512u * j));
+        };
+        auto issue_mmas = [&](int i, int s) {   // lane 0
+            const uint32_t st = stage_addr(s);
+            const uint32_t sf = sf_col(s);
+            constexpr uint32_t idesc = idesc_nvf4(kBM, BQ);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                tc_mma_nvf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + kOffQ + 32 * j), idesc,
+                            sf + 4 * j, sf + 16 + 4 * j, (i > 0 || j > 0) ? 1u : 0u);
+            tc_commit(empty_bar(s));   // frees the stage and its TMEM scale buffer
+        };
+        auto fence_and_sync = [&]() {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (lane == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tc_copy_32x128b_x4(col + 4 * j, desc_scale_atom(base + 512u * j));
-            }
         };
-        auto sf_col = [&](int s) { return tmem + (uint32_t)(C::ACC_COLS + s * C::SF_STRIDE); };
         const int first = min(nkt, S);
         bool ok = true;
         if (!prm.prefetch_w) grid_dependency_wait();
@@ -239,29 +249,49 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         // dependency when the weights were requested early).
         for (int i = 0; i < first && ok; ++i) {
             ok = warp_wait(wfull_bar(i), 0);
-            if (ok) atoms_to_tmem(stage_addr(i) + kWScaleOff, sf_col(i) + kWCol);
+            if (ok) build_atoms(stage_addr(i) + kWScaleOff);
+        }
+        if (ok) {
+            fence_and_sync();
+            if (lane == 0) {
+                tc_fence_after();
+                for (int i = 0; i < first; ++i) copy_atoms(stage_addr(i) + kWScaleOff, sf_col(i) + kWCol);
+            }
         }
         if (prm.prefetch_w) grid_dependency_wait();
-        constexpr uint32_t idesc = idesc_nvf4(kBM, BQ);
-        for (int i = 0; i < nkt && ok; ++i) {
+        // First pass: every resident K tile's token scales once they have
+        // all landed, one fence, then all copies and MMAs back to back.
+        for (int i = 0; i < first && ok; ++i) {
+            ok = warp_wait(tfull_bar(i), 0);
+            if (ok) build_atoms(stage_addr(i) + kTScaleOff);
+        }
+        if (ok) {
+            fence_and_sync();
+            if (lane == 0) {
+                tc_fence_after();
+                for (int i = 0; i < first; ++i) {
+                    copy_atoms(stage_addr(i) + kTScaleOff, sf_col(i) + kTCol);
+                    issue_mmas(i, i);
+                }
+            }
+            __syncwarp();
+        }
+        // Later K tiles (ring reuse): one at a time.
+        for (int i = first; i < nkt && ok; ++i) {
             const int s = i % S;
             const uint32_t ph = (uint32_t)(i / S) & 1u;
-            if (i >= first) {
-                ok = warp_wait(wfull_bar(s), ph);
-                if (!ok) break;
-                atoms_to_tmem(stage_addr(s) + kWScaleOff, sf_col(s) + kWCol);
-            }
+            ok = warp_wait(wfull_bar(s), ph);
+            if (!ok) break;
+            build_atoms(stage_addr(s) + kWScaleOff);
             ok = warp_wait(tfull_bar(s), ph);
             if (!ok) break;
-            atoms_to_tmem(stage_addr(s) + kTScaleOff, sf_col(s) + kTCol);
+            build_atoms(stage_addr(s) + kTScaleOff);
+            fence_and_sync();
             if (lane == 0) {
-                const uint32_t st = stage_addr(s);
-                const uint32_t sf = sf_col(s);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tc_mma_nvf4(tmem, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + kOffQ + 32 * j), idesc,
-                                sf + 4 * j, sf + 16 + 4 * j, (i > 0 || j > 0) ? 1u : 0u);
-                tc_commit(empty_bar(s));   // frees the stage and its TMEM scale buffer
+                tc_fence_after();
+                copy_atoms(stage_addr(s) + kWScaleOff, sf_col(s) + kWCol);
+                copy_atoms(stage_addr(s) + kTScaleOff, sf_col(s) + kTCol);
+                issue_mmas(i, s);
             }
             __syncwarp();
         }
