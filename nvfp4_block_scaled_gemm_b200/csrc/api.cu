@@ -481,6 +481,8 @@ bool pair_kernel_enabled() {
 // 4.3); M >= 8 loses.  NVFP4_GEMM_GEMV=0 turns the kernel off;
 // NVFP4_GEMM_GEMV=<n> (1..16) sends every M <= n to it (tuning and tests);
 // NVFP4_GEMM_GEMV_RW=1|2|4 forces the weight rows per CTA.
+bool use_gemv_areg(int M, int K);
+
 bool use_gemv(int M, int N, int K) {
     if (plan_override().set) return false;
     if (const char* e = std::getenv("NVFP4_GEMM_GEMV")) {
@@ -488,6 +490,7 @@ bool use_gemv(int M, int N, int K) {
         return M <= (v < 0 ? 0 : v > 16 ? 16 : v);
     }
     if (M == 1) return true;
+    if (M == 2 && use_gemv_areg(M, K)) return true;   // 8192 x 8192: 13.1 against 15.1 us
     if (K < 4096) return false;
     return (M == 2 && N <= 4096) || (M <= 4 && N <= 1024);
 }
@@ -536,6 +539,68 @@ nvfp4_status launch_gemv_rw(DeviceInfo* info, int rw, const nvfp4::GemvParams& p
     }
 }
 
+// The one-or-two-row form with the token chunks held in registers
+// (nvfp4_gemv_areg_kernel): M <= 2 and at most four chunks per thread for one
+// row (K <= 16384), two for two rows (K <= 8192).  NVFP4_GEMV_AREG=0 turns it
+// off (the general kernel then runs).
+template <int MT, int RW, int CPT>
+nvfp4_status launch_gemv_areg(DeviceInfo* info, const nvfp4::GemvParams& prm, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemv_areg_kernel<MT, RW, CPT>;
+    static const int per_sm = [kern] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, nvfp4::kGemvThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            b = 0;
+        }
+        return b > 0 ? b : 1;
+    }();
+    const int groups = (prm.N + RW - 1) / RW;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(groups, per_sm * info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+template <int MT, int CPT>
+nvfp4_status launch_gemv_areg_rw(DeviceInfo* info, int rw, const nvfp4::GemvParams& prm, cudaStream_t stream) {
+    switch (rw) {
+        case 1: return launch_gemv_areg<MT, 1, CPT>(info, prm, stream);
+        case 2: return launch_gemv_areg<MT, 2, CPT>(info, prm, stream);
+        default: return launch_gemv_areg<MT, 4, CPT>(info, prm, stream);
+    }
+}
+
+bool use_gemv_areg(int M, int K) {
+    if (const char* e = std::getenv("NVFP4_GEMV_AREG"))
+        if (e[0] == '0' && e[1] == '\0') return false;
+    const int cpt = (K / 32 + nvfp4::kGemvThreads - 1) / nvfp4::kGemvThreads;
+    return M >= 1 && M <= 2 && M * cpt <= 4;
+}
+
+nvfp4_status gemv_areg_gemm(DeviceInfo* info, int rw, const nvfp4::GemvParams& prm, cudaStream_t stream) {
+    const int cpt = (prm.K / 32 + nvfp4::kGemvThreads - 1) / nvfp4::kGemvThreads;
+    if (prm.M == 1) {
+        if (cpt <= 1) return launch_gemv_areg_rw<1, 1>(info, rw, prm, stream);
+        if (cpt <= 2) return launch_gemv_areg_rw<1, 2>(info, rw, prm, stream);
+        return launch_gemv_areg_rw<1, 4>(info, rw, prm, stream);
+    }
+    if (cpt <= 1) return launch_gemv_areg_rw<2, 1>(info, rw, prm, stream);
+    return launch_gemv_areg_rw<2, 2>(info, rw, prm, stream);
+}
+
 // The CUDA-core path for M <= 16.  Weight rows per CTA (measured): one row
 // for a single token row and a small matrix (spread over the most CTAs),
 // four from N = 2048 up, two with two or more token rows (each decoded
@@ -554,10 +619,17 @@ nvfp4_status gemv_gemm(DeviceInfo* info, const void* A, const void* sA, const vo
     prm.K = K;
     prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
     int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
+    if (use_gemv_areg(M, K)) {
+        // measured (us, 1 row): 2048 x 6144 rw2 2.53 / rw4 2.68; 8192 x 8192
+        // rw4 8.16 / rw2 8.27; 768 x 6144 rw1 1.94 / rw2 2.11.  Two rows:
+        // 256 x 6144 rw1 2.16 / rw2 2.39; 8192 x 8192 rw4 13.1 / rw2 14.6.
+        rw = N >= 4096 ? 4 : (M == 1 ? (N >= 2048 ? 2 : 1) : (N <= 256 ? 1 : 2));
+    }
     if (const char* e = std::getenv("NVFP4_GEMM_GEMV_RW")) {
         const int v = std::atoi(e);
         if (v == 1 || v == 2 || v == 4) rw = v;
     }
+    if (use_gemv_areg(M, K)) return gemv_areg_gemm(info, rw, prm, stream);
     if (M <= 1) return launch_gemv_rw<1>(info, rw, prm, stream);
     if (M <= 2) return launch_gemv_rw<2>(info, rw, prm, stream);
     if (M <= 4) return launch_gemv_rw<4>(info, rw, prm, stream);
@@ -791,9 +863,12 @@ SkPlan make_sk_plan(int M, int N, int K, const DeviceInfo* info) {
     // calls, constant weights): this kernel is faster up to 16 token rows
     // (768 x 6144: 5.3 against 6.1 us; 2048 x 6144: 6.9 against 7.8;
     // 256 x 6144: 4.5 against 5.7) and for 64 rows against 256 weight rows;
-    // beyond that the tiled kernel's deeper K pipeline wins.
-    if (f_swap < 0 && !(M <= 16 || (M <= 64 && N <= 256))) return p;
+    // beyond that the tiled kernel's deeper K pipeline wins.  It also loses
+    // with many weight tiles or a short K (8192 x 8192: 20.0 against 13.0 us;
+    // 6144 x 768: 7.2 against 5.5), so it takes at most 2048 weight rows and
+    // K >= 2048.
     const int k_tiles = K / 256;
+    if (f_swap < 0 && !((M <= 16 || (M <= 64 && N <= 256)) && N <= 2048 && k_tiles >= 8)) return p;
     p.swap = f_swap >= 0 ? f_swap == 1 : M <= 64;
     if (p.swap) {
         p.bq = f_bq ? f_bq : (M <= 16 ? 16 : 32);

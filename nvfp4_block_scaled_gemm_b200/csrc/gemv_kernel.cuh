@@ -312,6 +312,157 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_kernel(const GemvPara
 }
 
 // ---------------------------------------------------------------------------
+// One or two token rows: the same work split and arithmetic with fewer
+// instructions per weight chunk, which is what bounds the kernel above on
+// large weight matrices (about 100 warp instructions per 32-value chunk and
+// row, issue ~60% busy, at 8192 x 8192).
+//   * Each thread's K chunks of the token rows (CPT of them: c = t + 128 j)
+//     are decoded once, before the first row group, and kept as f16x2 with
+//     their scales as fp32: the row groups only decode weights.
+//   * A weight chunk's two E4M3 scales become an f16x2 in one conversion
+//     (every E4M3 value is an f16 value), then two fp32 values.
+//   * All CPT chunks of every row of a group are loaded at once; the next
+//     group's loads are issued before this group's reduction and store.
+// The per-block arithmetic is the kernel above's (exact block sums, an exact
+// fp32 scale product, one fp32 fma per block, chunks in the same order per
+// thread, the same warp and CTA reduction), so the results are identical.
+__device__ __forceinline__ uint32_t ld_stream_b16(const void* p) {
+    unsigned short v;
+    asm volatile("ld.global.nc.L1::no_allocate.b16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+// Two E4M3 bytes (low byte: the first block) -> their exact values.
+__device__ __forceinline__ float2 e4m3x2_values(uint32_t two) {
+    uint32_t h;
+    const unsigned short v = (unsigned short)two;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Resident CTAs per SM asked of the register allocator: two token rows
+// (64 registers of decoded chunks) four, or three with 4-row groups; one row
+// five, up to two chunks per thread.
+template <int MT, int RW, int CPT>
+constexpr int gemv_areg_min_ctas() {
+    return MT == 2 ? (RW * CPT >= 8 ? 3 : 4) : (CPT <= 2 ? 4 : 1);
+}
+
+template <int MT, int RW, int CPT>
+__global__ void __launch_bounds__(kGemvThreads, gemv_areg_min_ctas<MT, RW, CPT>())
+    nvfp4_gemv_areg_kernel(const GemvParams prm) {
+    static_assert(MT * CPT <= 4, "token chunks held in registers");
+    constexpr int NV = RW * MT;
+    __shared__ float red[2][kGemvWarps][NV];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int kc = prm.K >> 5;
+    const size_t row_bytes = (size_t)prm.K >> 1;
+    const size_t srow_bytes = (size_t)prm.K >> 4;
+    const int M = prm.M;
+    const int group_stride = gridDim.x * RW;
+    // chunks this thread owns: t, t + 128, ... below kc
+    int nch = 0;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) nch += (t + j * kGemvThreads < kc) ? 1 : 0;
+
+    uint4 bq[CPT][RW];
+    uint32_t bs[CPT][RW];
+    auto load_group = [&](int n0) {
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int n = min(n0 + r, prm.N - 1);
+            const uint8_t* br = prm.B + (size_t)n * row_bytes + 16 * (size_t)t;
+            const uint8_t* bsr = prm.sB + (size_t)n * srow_bytes + 2 * (size_t)t;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                if (j < nch) {
+                    bq[j][r] = ld_stream_v4(br + 16 * (size_t)(j * kGemvThreads));
+                    bs[j][r] = ld_stream_b16(bsr + 2 * (size_t)(j * kGemvThreads));
+                } else {
+                    bq[j][r] = make_uint4(0u, 0u, 0u, 0u);
+                    bs[j][r] = 0u;
+                }
+            }
+        }
+    };
+
+    grid_launch_dependents();
+    int n0 = blockIdx.x * RW;
+    if (prm.prefetch_b) load_group(n0);   // only B is touched before the wait
+    grid_dependency_wait();
+
+    uint32_t ah[MT][CPT][16];
+    float sa[MT][CPT][2];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + j * kGemvThreads;
+            if (m < M && j < nch) {
+                decode_chunk(ld_cached_v4(prm.A + (size_t)m * row_bytes + 16 * (size_t)c), ah[m][j]);
+                const float2 v = e4m3x2_values(ld_cached_u16(prm.sA + (size_t)m * srow_bytes + 2 * (size_t)c));
+                sa[m][j][0] = v.x;
+                sa[m][j][1] = v.y;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ah[m][j][i] = 0u;
+                sa[m][j][0] = sa[m][j][1] = 0.0f;
+            }
+        }
+    if (!prm.prefetch_b) load_group(n0);
+
+    for (int it = 0; n0 < prm.N; n0 += group_stride, ++it) {
+        float acc[RW][MT];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            if (j >= nch) break;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                uint32_t bh[16];
+                decode_chunk(bq[j][r], bh);
+                const float2 sb = e4m3x2_values(bs[j][r]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m < M) {
+                        acc[r][m] = fmaf(block_dot(ah[m][j], bh), sa[m][j][0] * sb.x, acc[r][m]);
+                        acc[r][m] = fmaf(block_dot(ah[m][j] + 8, bh + 8), sa[m][j][1] * sb.y, acc[r][m]);
+                    }
+                }
+            }
+        }
+        // the next row group's chunks, in flight during this group's reduction and store
+        const int n_next = n0 + group_stride;
+        if (n_next < prm.N) load_group(n_next);
+
+        float v[NV];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) v[r * MT + m] = acc[r][m];
+        warp_reduce_scatter<NV>(v, lane);
+        float (*rb)[NV] = red[it & 1];
+        if (gemv_writer_lane<NV>(lane)) {
+#pragma unroll
+            for (int j = 0; j < (NV >= 32 ? NV / 32 : 1); ++j) rb[warp][gemv_reduced_index<NV>(lane, j)] = v[j];
+        }
+        __syncthreads();   // also orders group it's reads of red[it & 1] before group it + 2's writes
+        for (int i = t; i < NV; i += kGemvThreads) {
+            const int r = i / MT, m = i % MT;
+            if (m < M && n0 + r < prm.N) {
+                float s = rb[0][i];
+#pragma unroll
+                for (int w = 1; w < kGemvWarps; ++w) s += rb[w][i];
+                prm.D[(size_t)m * prm.N + n0 + r] = __float2bfloat16_rn(s * prm.alpha);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // MXFP4 (OCP microscaling: E2M1 values, one E8M0 scale 2^(byte - 127) per 32
 // values) for a handful of token rows, on the CUDA cores.  A 16-byte chunk of
 // codes is exactly one scale block, so each thread reads one scale byte per
