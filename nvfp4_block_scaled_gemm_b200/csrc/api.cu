@@ -669,6 +669,60 @@ nvfp4_status launch_gemv_sp24_kernel(DeviceInfo* info, const nvfp4::GemvSp24Para
     return NVFP4_OK;
 }
 
+// One or two token rows: nvfp4_gemv_sp24_areg_kernel (the token chunks held
+// in registers), with the same limits as the dense form.
+template <int MT, int RW, int CPT>
+nvfp4_status launch_gemv_sp24_areg(DeviceInfo* info, const nvfp4::GemvSp24Params& prm, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemv_sp24_areg_kernel<MT, RW, CPT>;
+    static const int per_sm = [kern] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, nvfp4::kGemvThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            b = 0;
+        }
+        return b > 0 ? b : 1;
+    }();
+    const int groups = (prm.N + RW - 1) / RW;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(groups, per_sm * info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+template <int MT, int CPT>
+nvfp4_status launch_gemv_sp24_areg_rw(DeviceInfo* info, int rw, const nvfp4::GemvSp24Params& prm,
+                                      cudaStream_t stream) {
+    switch (rw) {
+        case 1: return launch_gemv_sp24_areg<MT, 1, CPT>(info, prm, stream);
+        case 2: return launch_gemv_sp24_areg<MT, 2, CPT>(info, prm, stream);
+        default: return launch_gemv_sp24_areg<MT, 4, CPT>(info, prm, stream);
+    }
+}
+
+nvfp4_status gemv_sp24_areg_gemm(DeviceInfo* info, int rw, const nvfp4::GemvSp24Params& prm, cudaStream_t stream) {
+    const int cpt = (prm.K / 32 + nvfp4::kGemvThreads - 1) / nvfp4::kGemvThreads;
+    if (prm.M == 1) {
+        if (cpt <= 1) return launch_gemv_sp24_areg_rw<1, 1>(info, rw, prm, stream);
+        if (cpt <= 2) return launch_gemv_sp24_areg_rw<1, 2>(info, rw, prm, stream);
+        return launch_gemv_sp24_areg_rw<1, 4>(info, rw, prm, stream);
+    }
+    if (cpt <= 1) return launch_gemv_sp24_areg_rw<2, 1>(info, rw, prm, stream);
+    return launch_gemv_sp24_areg_rw<2, 2>(info, rw, prm, stream);
+}
+
 template <int MT>
 nvfp4_status launch_gemv_sp24_rw(DeviceInfo* info, int rw, const nvfp4::GemvSp24Params& prm, cudaStream_t stream) {
     if (rw == 1) return launch_gemv_sp24_kernel<MT, 1>(info, prm, stream);
@@ -1517,10 +1571,13 @@ extern "C" nvfp4_status nvfp4_gemm_sparse24(const void* A, const void* sA, const
         prm.K = K;
         prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
         int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
+        const bool areg = use_gemv_areg(M, K);
+        if (areg) rw = N >= 4096 ? 4 : (M == 1 ? (N >= 2048 ? 2 : 1) : (N <= 256 ? 1 : 2));
         if (const char* e = std::getenv("NVFP4_GEMM_GEMV_RW")) {
             const int v = std::atoi(e);
             if (v == 1 || v == 2 || v == 4) rw = v;
         }
+        if (areg) return gemv_sp24_areg_gemm(info, rw, prm, stream);
         if (M <= 1) return launch_gemv_sp24_rw<1>(info, rw, prm, stream);
         if (M <= 2) return launch_gemv_sp24_rw<2>(info, rw, prm, stream);
         if (M <= 4) return launch_gemv_sp24_rw<4>(info, rw, prm, stream);

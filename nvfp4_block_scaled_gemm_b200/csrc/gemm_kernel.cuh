@@ -241,32 +241,47 @@ __device__ __forceinline__ void reduce_from_workspace(const GemmParams& prm, int
     } else {
         // Item (token row r, 8 weight columns c8): two float4 per rank,
         // one 16-byte store of D[p][q .. q+7]; lanes take consecutive r.
+        // With up to four ranks a thread has two items' loads in flight (every
+        // rank's, issued together), halving the round trips to L2.
+        constexpr int U = S <= 4 ? 2 : 1;
         const int items = rows_per * (BQ / 8);
-        for (int it = t; it < items; it += 128) {
-            const int r = it % rows_per, c8 = it / rows_per;
-            float acc[8];
+        for (int base = t; base < items; base += 128 * U) {
+            float4 a[U][S], b[U][S];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-            float4 a[S], b[S];   // every rank's loads in flight at once, then the sums in rank order
+            for (int u = 0; u < U; ++u) {
+                const int it = base + 128 * u;
+                if (it < items) {
+                    const int r = it % rows_per, c8 = it / rows_per;
 #pragma unroll
-            for (int z = 0; z < S; ++z) {
-                const float4* blk = partial_block<BQ>(prm, z);
-                a[z] = blk[(2 * c8) * kBM + row0 + r];
-                b[z] = blk[(2 * c8 + 1) * kBM + row0 + r];
+                    for (int z = 0; z < S; ++z) {
+                        const float4* blk = partial_block<BQ>(prm, z);
+                        a[u][z] = blk[(2 * c8) * kBM + row0 + r];
+                        b[u][z] = blk[(2 * c8 + 1) * kBM + row0 + r];
+                    }
+                }
             }
 #pragma unroll
-            for (int z = 0; z < S; ++z) {
-                acc[0] += a[z].x, acc[1] += a[z].y, acc[2] += a[z].z, acc[3] += a[z].w;
-                acc[4] += b[z].x, acc[5] += b[z].y, acc[6] += b[z].z, acc[7] += b[z].w;
-            }
-            const int p = tp * kBM + row0 + r, q = q_row0 + 8 * c8;
-            if (p < prm.rows_p && q < prm.rows_q) {   // rows_q (= N) is a multiple of 8
-                uint4 w;
-                w.x = pack_bf16x2(acc[0] * prm.alpha, acc[1] * prm.alpha);
-                w.y = pack_bf16x2(acc[2] * prm.alpha, acc[3] * prm.alpha);
-                w.z = pack_bf16x2(acc[4] * prm.alpha, acc[5] * prm.alpha);
-                w.w = pack_bf16x2(acc[6] * prm.alpha, acc[7] * prm.alpha);
-                *reinterpret_cast<uint4*>(prm.D + (size_t)p * prm.ldd + q) = w;
+            for (int u = 0; u < U; ++u) {
+                const int it = base + 128 * u;
+                if (it >= items) break;
+                const int r = it % rows_per, c8 = it / rows_per;
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll
+                for (int z = 0; z < S; ++z) {   // rank order
+                    acc[0] += a[u][z].x, acc[1] += a[u][z].y, acc[2] += a[u][z].z, acc[3] += a[u][z].w;
+                    acc[4] += b[u][z].x, acc[5] += b[u][z].y, acc[6] += b[u][z].z, acc[7] += b[u][z].w;
+                }
+                const int p = tp * kBM + row0 + r, q = q_row0 + 8 * c8;
+                if (p < prm.rows_p && q < prm.rows_q) {   // rows_q (= N) is a multiple of 8
+                    uint4 w;
+                    w.x = pack_bf16x2(acc[0] * prm.alpha, acc[1] * prm.alpha);
+                    w.y = pack_bf16x2(acc[2] * prm.alpha, acc[3] * prm.alpha);
+                    w.z = pack_bf16x2(acc[4] * prm.alpha, acc[5] * prm.alpha);
+                    w.w = pack_bf16x2(acc[6] * prm.alpha, acc[7] * prm.alpha);
+                    *reinterpret_cast<uint4*>(prm.D + (size_t)p * prm.ldd + q) = w;
+                }
             }
         }
     }

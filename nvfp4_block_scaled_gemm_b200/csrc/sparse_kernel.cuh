@@ -220,6 +220,157 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_sp24_kernel(const Gem
     }
 }
 
+// The same selector in fewer operations: v = m | m << 4 puts fields 0 and 2
+// at bits 0-1 and 8-9 and, shifted by 2, fields 1 and 3 at bits 4-5 and
+// 12-13 (equal to gather_selector for all 256 bytes).
+__device__ __forceinline__ uint32_t gather_selector_fast(uint32_t m) {
+    const uint32_t v = m | (m << 4);
+    return (v & 0x0303u) | ((v << 2) & 0x3030u) | 0x4400u;
+}
+
+// One or two token rows (the counterpart of nvfp4_gemv_areg_kernel): each
+// thread's token chunks (packed codes) and their scales (as fp32) are loaded
+// once and kept in registers, a weight chunk's two scales are converted in one
+// instruction, and all CPT chunks of a row group are loaded at once, the next
+// group's before this group's reduction.  The kept-pair arithmetic and the
+// summation order are nvfp4_gemv_sp24_kernel's, so the results are identical.
+template <int MT, int RW, int CPT>
+__global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_sp24_areg_kernel(const GemvSp24Params prm) {
+    static_assert(MT * CPT <= 4, "token chunks held in registers");
+    constexpr int NV = RW * MT;
+    __shared__ float red[2][kGemvWarps][NV];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int kc = prm.K >> 5;
+    const size_t arow_bytes = (size_t)prm.K >> 1;
+    const size_t vrow_bytes = (size_t)prm.K >> 2;
+    const size_t srow_bytes = (size_t)prm.K >> 4;
+    const int M = prm.M;
+    const int group_stride = gridDim.x * RW;
+    int nch = 0;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) nch += (t + j * kGemvThreads < kc) ? 1 : 0;
+
+    uint2 bq[CPT][RW];
+    uint32_t bm[CPT][RW], bs[CPT][RW];
+    auto load_group = [&](int n0) {
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int n = min(n0 + r, prm.N - 1);
+            const uint8_t* vr = prm.Bv + (size_t)n * vrow_bytes + 8 * (size_t)t;
+            const uint8_t* mr = prm.Bm + (size_t)n * srow_bytes + 2 * (size_t)t;
+            const uint8_t* sr = prm.sB + (size_t)n * srow_bytes + 2 * (size_t)t;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                if (j < nch) {
+                    bq[j][r] = ld_stream_v2(vr + 8 * (size_t)(j * kGemvThreads));
+                    bm[j][r] = ld_stream_u16(mr + 2 * (size_t)(j * kGemvThreads));
+                    bs[j][r] = ld_stream_u16(sr + 2 * (size_t)(j * kGemvThreads));
+                } else {
+                    bq[j][r] = make_uint2(0u, 0u);
+                    bm[j][r] = 0x4444u;
+                    bs[j][r] = 0u;
+                }
+            }
+        }
+    };
+
+    grid_launch_dependents();
+    int n0 = blockIdx.x * RW;
+    if (prm.prefetch_b) load_group(n0);   // only B is touched before the wait
+    grid_dependency_wait();
+
+    uint4 aq[MT][CPT];
+    float sa[MT][CPT][2];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + j * kGemvThreads;
+            if (m < M && j < nch) {
+                aq[m][j] = ld_cached_v4(prm.A + (size_t)m * arow_bytes + 16 * (size_t)c);
+                const float2 v = e4m3x2_values(ld_cached_u16(prm.sA + (size_t)m * srow_bytes + 2 * (size_t)c));
+                sa[m][j][0] = v.x;
+                sa[m][j][1] = v.y;
+            } else {
+                aq[m][j] = make_uint4(0u, 0u, 0u, 0u);
+                sa[m][j][0] = sa[m][j][1] = 0.0f;
+            }
+        }
+    if (!prm.prefetch_b) load_group(n0);
+
+    for (int it = 0; n0 < prm.N; n0 += group_stride, ++it) {
+        float acc[RW][MT];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            if (j >= nch) break;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const uint32_t sel01 = gather_selector_fast(bm[j][r] & 0xFFu);
+                const uint32_t sel23 = gather_selector_fast((bm[j][r] >> 8) & 0xFFu);
+                uint32_t bh[8], h4[4];
+                e2m1x8_to_f16x2(bq[j][r].x, h4);
+                bh[0] = h4[0], bh[1] = h4[1], bh[2] = h4[2], bh[3] = h4[3];
+                e2m1x8_to_f16x2(bq[j][r].y, h4);
+                bh[4] = h4[0], bh[5] = h4[1], bh[6] = h4[2], bh[7] = h4[3];
+                const float2 sb = e4m3x2_values(bs[j][r]);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m < M) {
+                        uint32_t ah[8], t4[4];
+                        e2m1x8_to_f16x2(__byte_perm(aq[m][j].x, aq[m][j].y, sel01), t4);
+                        ah[0] = t4[0], ah[1] = t4[1], ah[2] = t4[2], ah[3] = t4[3];
+                        e2m1x8_to_f16x2(__byte_perm(aq[m][j].z, aq[m][j].w, sel23), t4);
+                        ah[4] = t4[0], ah[5] = t4[1], ah[6] = t4[2], ah[7] = t4[3];
+                        float bsum[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t* a = ah + 4 * h;
+                            const uint32_t* w = bh + 4 * h;
+                            __half2 s2 = __hmul2(*reinterpret_cast<const __half2*>(&a[0]),
+                                                 *reinterpret_cast<const __half2*>(&w[0]));
+#pragma unroll
+                            for (int i = 1; i < 4; ++i)
+                                s2 = __hfma2(*reinterpret_cast<const __half2*>(&a[i]),
+                                             *reinterpret_cast<const __half2*>(&w[i]), s2);
+                            bsum[h] = __low2float(s2) + __high2float(s2);
+                        }
+                        acc[r][m] = fmaf(bsum[0], sa[m][j][0] * sb.x, acc[r][m]);
+                        acc[r][m] = fmaf(bsum[1], sa[m][j][1] * sb.y, acc[r][m]);
+                    }
+                }
+            }
+        }
+        const int n_next = n0 + group_stride;
+        if (n_next < prm.N) load_group(n_next);
+
+        float v[NV];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) v[r * MT + m] = acc[r][m];
+        warp_reduce_scatter<NV>(v, lane);
+        float (*rb)[NV] = red[it & 1];
+        if (gemv_writer_lane<NV>(lane)) {
+#pragma unroll
+            for (int q = 0; q < (NV >= 32 ? NV / 32 : 1); ++q) rb[warp][gemv_reduced_index<NV>(lane, q)] = v[q];
+        }
+        __syncthreads();
+        for (int e = t; e < NV; e += kGemvThreads) {
+            const int r = e / MT, m = e % MT;
+            if (m < M && n0 + r < prm.N) {
+                float sum = rb[0][e];
+#pragma unroll
+                for (int w = 1; w < kGemvWarps; ++w) sum += rb[w][e];
+                prm.D[(size_t)m * prm.N + n0 + r] = __float2bfloat16_rn(sum * prm.alpha);
+            }
+        }
+    }
+}
+
 // Kept bytes and position nibbles -> dense packed codes, one metadata byte
 // (two groups, 8 dense bytes) per item.
 __global__ void sparse24_expand_kernel(const uint8_t* __restrict__ values, const uint8_t* __restrict__ meta,

@@ -84,6 +84,45 @@ def test_sparse24_random_layout_every_instance(nv, monkeypatch, rw, M):
     assert not violations(run(nv, ca, sa, bv, bm, sb, alpha), ref, ad).any()
 
 
+@pytest.mark.parametrize("b_constant", [False, True])
+@pytest.mark.parametrize("M,N,K,rw", [
+    (1, 768, 6144, ""),      # 1.5 chunks per thread
+    (1, 8192, 8192, ""),     # 2 chunks per thread, 4-row groups
+    (1, 264, 16384, "2"),    # 4 chunks per thread
+    (2, 1000, 8192, "4"),    # two rows at their largest K; 250 groups of 4
+    (2, 136, 320, "1"),      # 10 chunks: most threads idle
+    (1, 8, 64, "1"),         # one chunk, half used
+])
+def test_sparse24_register_form_equals_general_kernel(nv, monkeypatch, M, N, K, rw, b_constant):
+    # One or two token rows run nvfp4_gemv_sp24_areg_kernel (token chunks held
+    # in registers); NVFP4_GEMV_AREG=0 runs nvfp4_gemv_sp24_kernel.  Same
+    # arithmetic and order: identical bits, and both within the oracle bound.
+    monkeypatch.delenv("NVFP4_GEMM_SP24_GEMV", raising=False)
+    monkeypatch.delenv("NVFP4_GEMV_AREG", raising=False)
+    if rw:
+        monkeypatch.setenv("NVFP4_GEMM_GEMV_RW", rw)
+    else:
+        monkeypatch.delenv("NVFP4_GEMM_GEMV_RW", raising=False)
+    rng = np.random.default_rng(2300 + M + N)
+    ca = synth.random_codes(M, K, 2301 + N)
+    sa = synth.random_scales(M, K, 2302 + N, lo=0x20, hi=0x40)
+    bv = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    pairs = np.array([0 | 1 << 2, 0 | 2 << 2, 0 | 3 << 2, 1 | 2 << 2, 1 | 3 << 2, 2 | 3 << 2], np.uint8)
+    nib = pairs[rng.integers(0, 6, size=(N, K // 8))]
+    bm = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    sb = synth.random_scales(N, K, 2303 + N, lo=0x20, hi=0x40)
+    alpha = 1.5e-3
+    _, ref, ad = oracle.gemm_sparse24(ca, sa, bv, bm, sb, alpha, M, N, K)
+    args = (dev(ca), dev(sa), dev(bv), dev(bm), dev(sb), alpha)
+    D = nv.gemm_sparse24(*args, b_constant=b_constant)
+    monkeypatch.setenv("NVFP4_GEMV_AREG", "0")
+    G = nv.gemm_sparse24(*args, b_constant=b_constant)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    assert torch.equal(D.view(torch.int16), G.view(torch.int16))
+    assert not violations(D.float().cpu().numpy(), ref, ad).any()
+
+
 def test_sparse24_equals_dense_gemm_on_expanded_weights(nv, monkeypatch):
     # Above the CUDA-core limit the entry point is the dense GEMM of the
     # expanded weights: the same bits as nvfp4_gemm on the oracle's expansion.
