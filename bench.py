@@ -397,7 +397,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(achieved / hbm_gbs, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} hbm_gbs",
-                     "kernel": "the GEMM launches of the step (one per GEMM; see DESIGN section 7)",
+                     "kernel": "the GEMM launches of the step (one per GEMM: the CUDA-core kernel at M = 1, split-K kernel at M = 16, tiled kernel above)",
                      "per_launch": {"algorithmic_bytes": bytes_per_launch, "avg_us": round(avg_launch_us, 3)}},
         "e2e": e2e,
         "gpu_launches": launches_per_rank,

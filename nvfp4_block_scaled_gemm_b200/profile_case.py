@@ -6,7 +6,7 @@
 `--traffic-csv FILE` (no GPU) instead turns the CSV log of an ncu run of
 `--shapes attn --iters 2` with the metrics gpu__time_duration.sum,
 dram__bytes_read.sum and dram__bytes_write.sum on the GEMM kernels
-(nvfp4_gemm_kernel, and nvfp4_gemv_kernel for M = 1) into the per-launch DRAM
+(every kernel named nvfp4_gemm_* or nvfp4_gemv_*) into the per-launch DRAM
 summary that bench.py reports as `roofline.traffic`
 (profiles/traffic_attn_sweep.json), stamped with the hash of the kernel code
 it was taken on.
@@ -42,6 +42,7 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
     last of the `iters` launches of each shape, in sweep order)."""
     import csv
     import json
+    import re
 
     from nvfp4_block_scaled_gemm_b200.build import source_hash
 
@@ -49,9 +50,11 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
         lines = [ln for ln in f if ln.startswith('"')]
     launches = {}
     for row in csv.DictReader(lines):
-        if not any(k in row["Kernel Name"] for k in ("nvfp4_gemm_kernel", "nvfp4_gemv_kernel")):
+        name = re.search(r"nvfp4_gem[mv]_\w*", row["Kernel Name"])
+        if not name:
             continue
         rec = launches.setdefault(int(row["ID"]), {})
+        rec["kernel"] = name.group(0)
         unit = row["Metric Unit"].strip().lower()
         val = float(row["Metric Value"].replace(",", ""))
         scale = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "ns": 1e-3, "nsecond": 1e-3, "us": 1.0,
@@ -61,15 +64,17 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
     shapes = parse_shapes("attn")
     if len(ids) != iters * len(shapes):
         raise SystemExit(f"expected {iters * len(shapes)} GEMM launches in {csv_path}, found {len(ids)}")
-    per_read, per_write, per_us = {}, {}, {}
+    per_read, per_write, per_us, per_kernel = {}, {}, {}, {}
     for i, (m, _, _) in enumerate(shapes):
         rec = launches[ids[iters * i + iters - 1]]
+        per_kernel[f"M{m}"] = rec["kernel"]
         per_read[f"M{m}"] = int(rec["dram__bytes_read.sum"])
         per_write[f"M{m}"] = int(rec["dram__bytes_write.sum"])
         per_us[f"M{m}"] = round(rec["gpu__time_duration.sum"], 2)
     mean = sum(per_read[k] + per_write[k] for k in per_read) / len(per_read)
     out = {
-        "kernel": "nvfp4_gemv_kernel (M = 1), nvfp4_gemm_kernel (the other five)",
+        "kernel": "the GEMM launch of each shape (per_shape_kernel)",
+        "per_shape_kernel": per_kernel,
         "workload": "attention sweep M in {1,16,64,128,256,512}, N=768, K=6144",
         "dram_bytes_per_launch": int(round(mean)),
         "per_shape_dram_read": per_read,
@@ -77,7 +82,7 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
         "per_shape_us_under_ncu": per_us,
         "source_hash": source_hash(),
         "command": "ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum "
-                   "--clock-control none -k regex:nvfp4_gem[mv]_kernel --csv --log-file traffic_attn.csv "
+                   "--clock-control none -k regex:nvfp4_gem --csv --log-file traffic_attn.csv "
                    "python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes attn --iters 2",
     }
     with open(out_path, "w") as f:
