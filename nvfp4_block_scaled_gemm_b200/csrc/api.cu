@@ -1116,6 +1116,21 @@ nvfp4_status launch_mx_by_bq(int bq, DeviceInfo* info, const Maps& m, const Gemm
     }
 }
 
+// The row-major-scale (SFR) MXFP4 instances: bits 20.. of the MX attribute mask.
+template <bool SWAP, bool SPLITK>
+nvfp4_status launch_mx_sfr_by_bq(int bq, DeviceInfo* info, const Maps& m, const GemmParams& prm, dim3 grid,
+                                 cudaStream_t stream) {
+    const int base = 20 + (SWAP ? 1 : 0) * 10 + (SPLITK ? 5 : 0);
+    switch (bq) {
+        case 16: return launch_gemm_kernel<16, SWAP, SPLITK, true, false, true>(info, 1ull << (base + 0), m, prm, grid, stream);
+        case 32: return launch_gemm_kernel<32, SWAP, SPLITK, true, false, true>(info, 1ull << (base + 1), m, prm, grid, stream);
+        case 64: return launch_gemm_kernel<64, SWAP, SPLITK, true, false, true>(info, 1ull << (base + 2), m, prm, grid, stream);
+        case 128: return launch_gemm_kernel<128, SWAP, SPLITK, true, false, true>(info, 1ull << (base + 3), m, prm, grid, stream);
+        case 256: return launch_gemm_kernel<256, SWAP, SPLITK, true, false, true>(info, 1ull << (base + 4), m, prm, grid, stream);
+        default: return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    }
+}
+
 nvfp4_status launch_swizzle_mx(const void* s, int rows, int K, void* out, cudaStream_t stream) {
     const int pairs = (K / 64 + 1) / 2;
     const long long lines = (long long)((rows + 127) / 128) * pairs * 32;
@@ -1761,8 +1776,41 @@ extern "C" nvfp4_status nvfp4_gemm_mxfp4(const void* A, const void* sA, const vo
         if (M == 2) return launch_gemv_mx_kernel<2, 2>(info, prm, stream);
         return launch_gemv_mx_kernel<4, 2>(info, prm, stream);
     }
-    // The tensor cores: both operands' scales re-laid out into atoms in
-    // per-stream scratch, then the tiled kernel's kind::mxf4 form.
+    // The tensor cores.  Row-major scales that TMA can load (K % 512 == 0, so
+    // that a row of K/32 scale bytes is a multiple of 16; 16-byte aligned):
+    // the tiled kernel lays them out on chip, as for NVFP4.  Otherwise both
+    // operands' scales are first re-laid out into atoms in per-stream scratch.
+    const bool sfr = (K % 512 == 0) && aligned(sA, 16) && aligned(sB, 16) && !std::getenv("NVFP4_GEMM_MX_ATOMS");
+    if (sfr) {
+        const Plan plan = make_plan(M, N, K, info, /*sfr=*/true);
+        const void* P = plan.swap ? B : A;
+        const void* Q = plan.swap ? A : B;
+        const void* sP = plan.swap ? sB : sA;
+        const void* sQ = plan.swap ? sA : sB;
+        const int rows_p = plan.swap ? N : M;
+        const int rows_q = plan.swap ? M : N;
+        Maps maps;
+        if (!make_operand_map(&maps.p, P, rows_p, K / 2, 128) || !make_operand_map(&maps.q, Q, rows_q, K / 2, plan.bq) ||
+            !make_scale_map(&maps.sp, sP, rows_p, K / 32, 128) || !make_scale_map(&maps.sq, sQ, rows_q, K / 32, plan.bq))
+            return NVFP4_ERR_CUDA;
+        GemmParams prm{};
+        prm.D = static_cast<__nv_bfloat16*>(D);
+        prm.alpha = alpha;
+        prm.rows_p = rows_p;
+        prm.rows_q = rows_q;
+        prm.K = K;
+        prm.ldd = N;
+        prm.k_tiles = plan.k_tiles;
+        prm.tiles_q = plan.tiles_q;
+        prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+        if ((st = splitk_ws(dev, stream, plan, nullptr, 0, &prm.ws)) != NVFP4_OK) return st;
+        const dim3 grid(plan.splits, plan.tiles_q * plan.tiles_p, 1);
+        if (plan.swap)
+            return plan.splits > 1 ? launch_mx_sfr_by_bq<true, true>(plan.bq, info, maps, prm, grid, stream)
+                                   : launch_mx_sfr_by_bq<true, false>(plan.bq, info, maps, prm, grid, stream);
+        return plan.splits > 1 ? launch_mx_sfr_by_bq<false, true>(plan.bq, info, maps, prm, grid, stream)
+                               : launch_mx_sfr_by_bq<false, false>(plan.bq, info, maps, prm, grid, stream);
+    }
     const Plan plan = make_plan(M, N, K, info, /*sfr=*/false);
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;

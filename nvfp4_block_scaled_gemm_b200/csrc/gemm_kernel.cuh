@@ -157,6 +157,14 @@ __device__ __forceinline__ void gather_scale_words(uint32_t base, int lane, uint
     }
 }
 
+// MXFP4 row-major scale box (16 bytes = two K tiles per row): move the words
+// of the second K tile (2, 3) into the places of the first (0, 1) when `hi`.
+// out[4 w + r1] is word w of row group r1, as gather_scale_words leaves it.
+__device__ __forceinline__ void mx_box_half(uint32_t (&w)[16], bool hi) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = hi ? w[i + 8] : w[i];
+}
+
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -287,17 +295,20 @@ __device__ __forceinline__ void reduce_from_workspace(const GemmParams& prm, int
     }
 }
 
-// MX: the MXFP4 form (E8M0 scale per 32 values, kind::mxf4 block32), with
-// scales pre-laid out in 512-byte atoms of two K steps each (non-SFR only):
-// the atoms of a K tile are two per 128-row block instead of four, and step j
-// reads TMEM scale word j / 2 at byte 2 * (j % 2).
+// MX: the MXFP4 form (E8M0 scale per 32 values, kind::mxf4 block32): a K
+// tile has 8 scale bytes per row, two TMEM words (steps 0-1, 2-3), and step
+// j reads word j / 2 at byte 2 * (j % 2).  Without SFR the scales come
+// pre-laid out in 512-byte atoms of two K steps each (two per 128-row block
+// and K tile).  With SFR they are row-major [rows][K/32] (K % 512 == 0): a
+// TMA box starts on a 16-byte boundary, so K tile kt loads the 16-byte box of
+// K tiles kt & ~1 and kt | 1, and the writers take its half kt % 2.
 template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false, bool MX = false>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                       const GemmParams prm) {
     static_assert(!QBF16 || (SWAP && SFR && BQ <= 64), "BF16 activations: swapped layout, row-major scale tiles");
-    static_assert(!MX || (!SFR && !QBF16), "MXFP4: pre-laid-out scale atoms");
+    static_assert(!MX || !QBF16, "MXFP4: FP4 activations");
     using C = TileConfig<BQ, SPLITK, QBF16>;
     constexpr int S = C::STAGES;
     constexpr int NB = kScaleBuffers;
@@ -375,6 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the CTAs of one wave and the column block Q by every wave.
             const uint64_t pol_p = SWAP ? policy_evict_first() : policy_evict_normal();
             const uint64_t pol_q = policy_evict_last();
+            // x (bytes) of K tile kt's row-major scale box: 16 scale bytes
+            // per K tile (NVFP4), or the 16 bytes of K tiles kt & ~1, kt | 1 (MXFP4)
+            auto sf_x = [](int kt) { return MX ? 16 * (kt >> 1) : 16 * kt; };
             // With a constant B, its first ring's worth of tiles is requested
             // before waiting for the previous grid (only B is touched then).
             // bytes of one stage: P tile + P scales + the Q side (FP4 tile and
@@ -386,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(st + C::QRAW_OFF, &tmQ, bar, kt * 256, q_row0, pol_q);
                 } else {
                     tma_load_2d(st + C::P_BYTES, &tmQ, bar, kt * kStageKBytes, q_row0, pol_q);
-                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, bar, kt * 16, q_row0, pol_q);
+                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, bar, sf_x(kt), q_row0, pol_q);
                 }
             };
             int pre = 0;
@@ -398,10 +412,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(full_bar(i), kStageTx);
                     if (SWAP) {   // B is P
                         tma_load_2d(st, &tmP, full_bar(i), kt * kStageKBytes, tp * kBM, pol_p);
-                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(i), kt * 16, tp * kBM, pol_p);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(i), sf_x(kt), tp * kBM, pol_p);
                     } else {      // B is Q
                         tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(i), kt * kStageKBytes, q_row0, pol_q);
-                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(i), kt * 16, q_row0,
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(i), sf_x(kt), q_row0,
                                     pol_q);
                     }
                 }
@@ -417,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         load_q(st, full_bar(s), kt);
                     } else {
                         tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
-                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
+                        tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), sf_x(kt), tp * kBM, pol_p);
                     }
                     continue;
                 }
@@ -426,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // row-major scale tiles: 16 bytes (= 4 K steps) per row
                     mbar_arrive_expect_tx(full_bar(s), kStageTx);
                     tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
-                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), kt * 16, tp * kBM, pol_p);
+                    tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), sf_x(kt), tp * kBM, pol_p);
                     load_q(st, full_bar(s), kt);
                 } else {
                     // atoms per 128-row block: one per K step (NVFP4) or per
@@ -555,12 +569,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int iu = it + u;
                     const uint32_t st = smem_base + (iu % S) * C::STAGE_BYTES;
                     const uint32_t sf = t_quad + C::SF_BASE + (iu % NB) * C::SF_STRIDE;
+                    // MXFP4 row-major: this K tile's two words are words 2h, 2h + 1 of the box
+                    const bool hi = MX && SFR && ((kt_begin + iu) & 1);
                     uint32_t wp[16];
                     gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES, lane, wp);
+                    mx_box_half(wp, hi);
                     tmem_store_16(sf, wp);
                     if (C::Q_BLOCKS == 1) {
                         uint32_t wq[16];
                         gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq);
+                        mx_box_half(wq, hi);
                         tmem_store_16(sf + 16, wq);
                     } else {
                         // two 128-row blocks: step j uses columns 8j + 4*block + r1
@@ -568,6 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, lane, wq0);
                         gather_scale_words<SFR>(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES + 4 * kAtomBytes, lane,
                                                 wq1);
+                        mx_box_half(wq0, hi);
+                        mx_box_half(wq1, hi);
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
 #pragma unroll

@@ -7,8 +7,11 @@ as random codes and scales; expected values come from oracle_gemm_mxfp4
 (an exact sum, rounded once), and every output must satisfy
     |gpu - ref| <= 2^-8 |ref| + 2^-20 |alpha| sum_k |a_k b_k|.
 Both paths run: the CUDA-core kernel for up to 4 token rows and the
-tensor-core kernel (kind::mxf4, scales re-laid out into atoms) above, the
-latter through every tile plan NVFP4_GEMM_PLAN can force.
+tensor-core kernel (kind::mxf4) above, the latter through every tile plan
+NVFP4_GEMM_PLAN can force and with both scale layouts: row-major tiles laid
+out on chip (K % 512 == 0; a TMA box covers two K tiles and the kernel takes
+its half) and, with NVFP4_GEMM_MX_ATOMS=1 or any other K, atoms re-laid out
+in scratch first.
 """
 import numpy as np
 import pytest
@@ -59,12 +62,23 @@ def test_mxfp4_decode_kernel(nv, M, N, K, kind, b_constant):
     check(nv, ca, sa, cb, sb, 0.75, M, N, K, b_constant)
 
 
+@pytest.fixture(params=["rowmajor", "atoms"])
+def layout(request, monkeypatch):
+    if request.param == "atoms":
+        monkeypatch.setenv("NVFP4_GEMM_MX_ATOMS", "1")
+    else:
+        monkeypatch.delenv("NVFP4_GEMM_MX_ATOMS", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("M,N,K,kind", [
     (5, 768, 6144, "normal"), (16, 2048, 2048, "moe"), (37, 264, 1024, "uniform"), (100, 520, 1024, "normal"),
-    (300, 136, 2048, "moe"), (200, 264, 320, "uniform"), (129, 8, 192, "normal"), (700, 1024, 512, "uniform")])
-def test_mxfp4_tensor_cores(nv, M, N, K, kind):
+    (300, 136, 2048, "moe"), (200, 264, 320, "uniform"), (129, 8, 192, "normal"), (700, 1024, 512, "uniform"),
+    (512, 768, 6144, "normal"), (64, 2048, 1536, "moe")])
+@pytest.mark.parametrize("b_constant", [False, True])
+def test_mxfp4_tensor_cores(nv, layout, M, N, K, kind, b_constant):
     ca, sa, cb, sb = mx_problem(M, N, K, kind, 900 + M + N + K)
-    check(nv, ca, sa, cb, sb, 1.0, M, N, K)
+    check(nv, ca, sa, cb, sb, 1.0, M, N, K, b_constant)
 
 
 @pytest.mark.parametrize("plan,M,N,K", [
@@ -73,8 +87,10 @@ def test_mxfp4_tensor_cores(nv, M, N, K, kind):
     ("0:128:2", 300, 520, 1024),  # unswapped, split
     ("0:256:1", 512, 512, 2048),  # 256-wide tiles: two 128-row scale blocks per Q tile
     ("1:16:1", 40, 264, 448),     # K % 128 == 64: the last atom holds one K step
+    ("1:32:8", 24, 256, 6144),    # 8-way split of 24 K tiles: slices start on odd K tiles too
+    ("0:64:8", 256, 512, 4096),   # unswapped 8-way split, row-major scales
 ])
-def test_mxfp4_forced_plans(nv, monkeypatch, plan, M, N, K):
+def test_mxfp4_forced_plans(nv, monkeypatch, layout, plan, M, N, K):
     monkeypatch.setenv("NVFP4_GEMM_PLAN", plan)
     monkeypatch.setenv("NVFP4_GEMM_GEMV", "0")
     ca, sa, cb, sb = mx_problem(M, N, K, "uniform", 1000 + M)
@@ -93,12 +109,13 @@ def test_mxfp4_random_codes_and_scales(nv, M):
     check(nv, ca, sa, cb, sb, 1.0 / 3.0, M, N, K)
 
 
-@pytest.mark.parametrize("M", [1, 24])
-def test_mxfp4_one_hot_pins_layout(nv, M):
+@pytest.mark.parametrize("M,K", [(1, 256), (24, 256), (24, 1024), (40, 2048)])
+def test_mxfp4_one_hot_pins_layout(nv, M, K):
     # A row of one-hot codes against scaled one-hot columns: each output is a
     # single exact product, which pins the nibble order and which E8M0 byte
-    # (block k / 32) scales element k, on both paths.
-    N, K = 64, 256
+    # (block k / 32) scales element k, on both paths; K = 1024 and 2048 run
+    # the row-major-scale form, whose odd K tiles read the upper half of a box.
+    N = 64
     rng = np.random.default_rng(5 + M)
     ka = rng.integers(0, K, M)
     kb = rng.integers(0, K, N)
