@@ -1146,6 +1146,46 @@ nvfp4_status launch_swizzle_mx(const void* s, int rows, int K, void* out, cudaSt
 
 size_t mx_atom_bytes(int rows, int K) { return (size_t)((rows + 127) / 128) * (size_t)((K / 64 + 1) / 2) * 512u; }
 
+template <int MT, int RW, int CPT>
+nvfp4_status launch_gemv_mx_areg(DeviceInfo* info, const nvfp4::GemvMxParams& prm, cudaStream_t stream) {
+    auto kern = nvfp4::nvfp4_gemv_mx_areg_kernel<MT, RW, CPT>;
+    static const int per_sm = [kern] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, nvfp4::kGemvThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            b = 0;
+        }
+        return b > 0 ? b : 1;
+    }();
+    const int groups = (prm.N + RW - 1) / RW;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(groups, per_sm * info->num_sms), 1, 1);
+    cfg.blockDim = dim3(nvfp4::kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    g_launches++;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
+}
+
+template <int MT, int CPT>
+nvfp4_status launch_gemv_mx_areg_rw(DeviceInfo* info, int rw, const nvfp4::GemvMxParams& prm, cudaStream_t stream) {
+    switch (rw) {
+        case 1: return launch_gemv_mx_areg<MT, 1, CPT>(info, prm, stream);
+        case 2: return launch_gemv_mx_areg<MT, 2, CPT>(info, prm, stream);
+        default: return launch_gemv_mx_areg<MT, 4, CPT>(info, prm, stream);
+    }
+}
+
 template <int MT, int RW>
 nvfp4_status launch_gemv_mx_kernel(DeviceInfo* info, const nvfp4::GemvMxParams& prm, cudaStream_t stream) {
     auto kern = nvfp4::nvfp4_gemv_mx_kernel<MT, RW>;
@@ -1771,6 +1811,21 @@ extern "C" nvfp4_status nvfp4_gemm_mxfp4(const void* A, const void* sA, const vo
         prm.N = N;
         prm.K = K;
         prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
+        if (use_gemv_areg(M, K)) {
+            int rw = N >= 4096 ? 4 : (M == 1 ? (N >= 2048 ? 2 : 1) : (N <= 256 ? 1 : 2));
+            if (const char* e = std::getenv("NVFP4_GEMM_GEMV_RW")) {
+                const int v = std::atoi(e);
+                if (v == 1 || v == 2 || v == 4) rw = v;
+            }
+            const int cpt = (K / 32 + nvfp4::kGemvThreads - 1) / nvfp4::kGemvThreads;
+            if (M == 1) {
+                if (cpt <= 1) return launch_gemv_mx_areg_rw<1, 1>(info, rw, prm, stream);
+                if (cpt <= 2) return launch_gemv_mx_areg_rw<1, 2>(info, rw, prm, stream);
+                return launch_gemv_mx_areg_rw<1, 4>(info, rw, prm, stream);
+            }
+            if (cpt <= 1) return launch_gemv_mx_areg_rw<2, 1>(info, rw, prm, stream);
+            return launch_gemv_mx_areg_rw<2, 2>(info, rw, prm, stream);
+        }
         const int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
         if (M == 1) return rw == 4 ? launch_gemv_mx_kernel<1, 4>(info, prm, stream) : launch_gemv_mx_kernel<1, 1>(info, prm, stream);
         if (M == 2) return launch_gemv_mx_kernel<2, 2>(info, prm, stream);

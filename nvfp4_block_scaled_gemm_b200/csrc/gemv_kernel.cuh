@@ -582,4 +582,125 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_mx_kernel(const GemvM
     }
 }
 
+// One or two token rows of MXFP4 (the counterpart of nvfp4_gemv_areg_kernel):
+// each thread's token chunks are decoded once and held in registers with
+// their E8M0 exponents, all CPT weight chunks of a row group are loaded at
+// once and the next group's before this group's reduction.  A chunk's exact
+// sum is scaled by 2^(ea + eb - 254) with one multiply while that power is a
+// normal fp32 number -- the same value ldexpf gives, exact unless the result
+// is subnormal, where both round to nearest even -- and by ldexpf otherwise;
+// the sums and their order are nvfp4_gemv_mx_kernel's, so the results are
+// identical.
+template <int MT, int RW, int CPT>
+__global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_mx_areg_kernel(const GemvMxParams prm) {
+    static_assert(MT * CPT <= 4, "token chunks held in registers");
+    constexpr int NV = RW * MT;
+    __shared__ float red[2][kGemvWarps][NV];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int kc = prm.K >> 5;
+    const size_t row_bytes = (size_t)prm.K >> 1;
+    const size_t srow_bytes = (size_t)prm.K >> 5;
+    const int M = prm.M;
+    const int group_stride = gridDim.x * RW;
+    int nch = 0;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) nch += (t + j * kGemvThreads < kc) ? 1 : 0;
+
+    uint4 bq[CPT][RW];
+    uint32_t bs[CPT][RW];
+    auto load_group = [&](int n0) {
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int n = min(n0 + r, prm.N - 1);
+            const uint8_t* br = prm.B + (size_t)n * row_bytes + 16 * (size_t)t;
+            const uint8_t* bsr = prm.sB + (size_t)n * srow_bytes + (size_t)t;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                if (j < nch) {
+                    bq[j][r] = ld_stream_v4(br + 16 * (size_t)(j * kGemvThreads));
+                    bs[j][r] = ld_stream_u8(bsr + (size_t)(j * kGemvThreads));
+                } else {
+                    bq[j][r] = make_uint4(0u, 0u, 0u, 0u);
+                    bs[j][r] = 127u;
+                }
+            }
+        }
+    };
+
+    grid_launch_dependents();
+    int n0 = blockIdx.x * RW;
+    if (prm.prefetch_b) load_group(n0);   // only B is touched before the wait
+    grid_dependency_wait();
+
+    uint32_t ah[MT][CPT][16];
+    int ea[MT][CPT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + j * kGemvThreads;
+            if (m < M && j < nch) {
+                decode_chunk(ld_cached_v4(prm.A + (size_t)m * row_bytes + 16 * (size_t)c), ah[m][j]);
+                ea[m][j] = (int)__ldg(prm.sA + (size_t)m * srow_bytes + (size_t)c);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ah[m][j][i] = 0u;
+                ea[m][j] = 127;
+            }
+        }
+    if (!prm.prefetch_b) load_group(n0);
+
+    for (int it = 0; n0 < prm.N; n0 += group_stride, ++it) {
+        float acc[RW][MT];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            if (j >= nch) break;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                uint32_t bh[16];
+                decode_chunk(bq[j][r], bh);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m < M) {
+                        const float blk = block_dot(ah[m][j], bh) + block_dot(ah[m][j] + 8, bh + 8);   // exact
+                        const int e = ea[m][j] + (int)bs[j][r] - 254;
+                        const float scaled = (e >= -126 && e <= 127)
+                                                 ? blk * __uint_as_float((uint32_t)(e + 127) << 23)
+                                                 : ldexpf(blk, e);
+                        acc[r][m] += scaled;
+                    }
+                }
+            }
+        }
+        const int n_next = n0 + group_stride;
+        if (n_next < prm.N) load_group(n_next);
+
+        float v[NV];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) v[r * MT + m] = acc[r][m];
+        warp_reduce_scatter<NV>(v, lane);
+        float (*rb)[NV] = red[it & 1];
+        if (gemv_writer_lane<NV>(lane)) {
+#pragma unroll
+            for (int q = 0; q < (NV >= 32 ? NV / 32 : 1); ++q) rb[warp][gemv_reduced_index<NV>(lane, q)] = v[q];
+        }
+        __syncthreads();
+        for (int e = t; e < NV; e += kGemvThreads) {
+            const int r = e / MT, m = e % MT;
+            if (m < M && n0 + r < prm.N) {
+                float sum = rb[0][e];
+#pragma unroll
+                for (int w = 1; w < kGemvWarps; ++w) sum += rb[w][e];
+                prm.D[(size_t)m * prm.N + n0 + r] = __float2bfloat16_rn(sum * prm.alpha);
+            }
+        }
+    }
+}
+
 }  // namespace nvfp4

@@ -133,6 +133,33 @@ def test_mxfp4_one_hot_pins_layout(nv, M, K):
     assert np.array_equal(got, oracle.bf16_bits_to_float(D))     # one exact product per output: bit-exact
 
 
+@pytest.mark.parametrize("M,N,K,scales", [
+    (1, 768, 6144, "moderate"), (2, 256, 6144, "moderate"), (1, 1032, 12288, "moderate"),
+    (2, 264, 8192, "moderate"), (1, 264, 2048, "tiny"), (2, 136, 1024, "tiny"), (1, 8, 64, "moderate")])
+@pytest.mark.parametrize("b_constant", [False, True])
+def test_mxfp4_register_form_equals_general_kernel(nv, monkeypatch, M, N, K, scales, b_constant):
+    # One or two token rows run nvfp4_gemv_mx_areg_kernel; NVFP4_GEMV_AREG=0
+    # runs nvfp4_gemv_mx_kernel.  Identical bits, both within the bound.
+    # "tiny": exponent sums ea + eb - 254 from -174 to -94, so chunks take both
+    # the multiply (a normal power of two) and the ldexpf branch.
+    monkeypatch.delenv("NVFP4_GEMV_AREG", raising=False)
+    rng = np.random.default_rng(3000 + M + N + K)
+    ca, cb = synth.random_codes(M, K, 3001 + N), synth.random_codes(N, K, 3002 + N)
+    lo, hi = (107, 140) if scales == "moderate" else (40, 81)
+    sa = rng.integers(lo, hi, size=(M, K // 32), dtype=np.uint8)
+    sb = rng.integers(lo, hi, size=(N, K // 32), dtype=np.uint8)
+    alpha = 0.375
+    _, ref, ad = oracle.gemm_mxfp4(ca, sa, cb, sb, alpha, M, N, K)
+    args = (dev(ca), dev(sa), dev(cb), dev(sb), alpha)
+    D = nv.gemm_mxfp4(*args, b_constant=b_constant)
+    monkeypatch.setenv("NVFP4_GEMV_AREG", "0")
+    G = nv.gemm_mxfp4(*args, b_constant=b_constant)
+    torch.cuda.synchronize()
+    assert nv.get_device_error() == 0
+    assert torch.equal(D.view(torch.int16), G.view(torch.int16))
+    assert not violations(D.float().cpu().numpy(), ref, ad).any()
+
+
 def test_mxfp4_deterministic_and_guarded(nv):
     M, N, K = 64, 768, 2048
     ca, sa, cb, sb = mx_problem(M, N, K, "moe", 1234)
