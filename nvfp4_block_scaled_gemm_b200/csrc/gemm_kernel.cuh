@@ -490,6 +490,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_commit(empty_bar(s));
                     continue;
                 }
+                if (MX && steps == 4) {
+                    // steps 2w and 2w + 1 share scale word w, bytes 0-1 and 2-3
+                    const uint64_t dp = desc_kmajor_sw128(st), dq = desc_kmajor_sw128(st + C::P_BYTES);
+                    constexpr uint32_t id0 = idesc_mxf4(kBM, BQ, 0), id2 = idesc_mxf4(kBM, BQ, 2);
+                    const uint32_t acc0 = it > 0 ? 1u : 0u;
+                    tc_mma_mxf4(tmem, dp, dq, id0, sf, sf + 16, acc0);
+                    tc_mma_mxf4(tmem, dp + 2u, dq + 2u, id2, sf, sf + 16, 1u);
+                    tc_mma_mxf4(tmem, dp + 4u, dq + 4u, id0, sf + 4, sf + 16 + 4 * C::Q_BLOCKS, 1u);
+                    tc_mma_mxf4(tmem, dp + 6u, dq + 6u, id2, sf + 4, sf + 16 + 4 * C::Q_BLOCKS, 1u);
+                    tc_commit(empty_bar(s));
+                    continue;
+                }
                 for (int j = 0; j < steps; ++j) {
                     if (MX) {
                         // the atoms' word (j / 2) landed in TMEM column group j / 2
