@@ -1012,8 +1012,16 @@ nvfp4_status launch_sk_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, con
     return NVFP4_OK;
 }
 
-nvfp4_status sk_gemm(DeviceInfo* info, const SkPlan& plan, const void* A, const void* sA, const void* B,
-                     const void* sB, float alpha, void* D, int M, int N, int K, unsigned flags, cudaStream_t stream) {
+// Split-K workspace of the split-K kernel: one fp32 partial tile per (tile, rank).
+size_t sk_ws_bytes(const SkPlan& p) {
+    return p.splits > 1 ? (size_t)p.tiles_p * p.tiles_q * p.splits * (size_t)p.bq * 128u * 4u : 0;
+}
+
+// `ws_fixed`: the caller-owned workspace of nvfp4_gemm_noalloc (at least
+// sk_ws_bytes(plan) bytes), else per-stream scratch.
+nvfp4_status sk_gemm(int dev, DeviceInfo* info, const SkPlan& plan, const void* A, const void* sA, const void* B,
+                     const void* sB, float alpha, void* D, int M, int N, int K, unsigned flags, cudaStream_t stream,
+                     uint8_t* ws_fixed = nullptr) {
     const void* P = plan.swap ? B : A;
     const void* Q = plan.swap ? A : B;
     const void* sP = plan.swap ? sB : sA;
@@ -1035,6 +1043,15 @@ nvfp4_status sk_gemm(DeviceInfo* info, const SkPlan& plan, const void* A, const 
     prm.stages = plan.stages;
     prm.prefetch_w = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
     prm.tmem_cols = plan.tmem_cols;
+    const size_t ws_bytes = sk_ws_bytes(plan);
+    if (ws_bytes > 0) {
+        uint8_t* ws = ws_fixed;
+        if (ws == nullptr) {
+            const nvfp4_status st = get_scratch(dev, stream, ws_bytes, &ws, kScratchSplitK);
+            if (st != NVFP4_OK) return st;
+        }
+        prm.ws = reinterpret_cast<float4*>(ws);
+    }
     if (plan.swap) {
         switch (plan.bq) {
             case 16: return launch_sk_kernel<16, true>(info, 1ull << 50, maps, prm, plan, stream);
@@ -1057,7 +1074,8 @@ nvfp4_status sfr_gemm(int dev, DeviceInfo* info, Plan plan, const void* A, const
                       cudaStream_t stream, uint8_t* ws_fixed = nullptr, size_t ws_cap = 0) {
     if (!plan_override().set) {
         const SkPlan sk = make_sk_plan(M, N, K, info);
-        if (sk.use) return sk_gemm(info, sk, A, sA, B, sB, alpha, D, M, N, K, flags, stream);
+        if (sk.use && (ws_fixed == nullptr || sk_ws_bytes(sk) <= ws_cap))
+            return sk_gemm(dev, info, sk, A, sA, B, sB, alpha, D, M, N, K, flags, stream, ws_fixed);
     }
     if (ws_fixed != nullptr && splitk_ws_bytes(plan) > ws_cap) plan = make_plan(M, N, K, info, true, 1);
     const void* P = plan.swap ? B : A;

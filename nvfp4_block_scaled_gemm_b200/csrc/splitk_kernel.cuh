@@ -23,12 +23,11 @@
 //     and the weight scales are moved into TMEM before it as well.  After the
 //     wait only the activation tiles (a few KB), their scales, the MMAs and
 //     the split-K reduction remain.
-//   * The split-K partials meet in distributed shared memory: each CTA sends
-//     the fp32 rows of its 128 x BQ partial straight from registers to the
-//     rank that owns them (st.async, counted in bytes on the owner's
-//     mbarrier, so no cluster-wide barrier is needed after the exchange), and
-//     the owner sums its rows over the ranks in rank order (deterministic)
-//     and writes them with 16-byte stores.
+//   * The split-K partials meet in L2: each CTA writes its fp32 128 x BQ
+//     partial to a global workspace with coalesced 16-byte stores, one
+//     cluster barrier (release/acquire at cluster scope) makes them visible,
+//     and each rank sums its 128 / splits rows over the ranks in rank order
+//     (deterministic) and writes them with 16-byte stores.
 //
 // Orientation.  SWAP (token rows <= 64): the weights are the 128-row MMA
 // operand P and the token rows the BQ-wide operand Q (BQ = 16, 32, 64); the
@@ -50,8 +49,8 @@
 // this kernel is chosen for, a CTA's whole K slice usually fits, so nothing
 // is reused.  Barriers per stage: wfull (weight tile and scales landed),
 // tfull (token tile and scales landed), empty (the MMA commit: stage and
-// TMEM scale buffer free); plus accum (all MMAs done) and red (all ranks'
-// partial rows for this CTA have arrived).  Every wait is bounded.
+// TMEM scale buffer free); plus accum (all MMAs done).  Every wait is
+// bounded.
 #pragma once
 
 #include "gemm_kernel.cuh"
@@ -69,8 +68,6 @@ struct SkConfig {
     static constexpr int SFP_BYTES = 2048;                   // 128 rows x 16 scale bytes
     static constexpr int SFQ_BYTES = 2048;                   // BQ <= 128 rows x 16 scale bytes
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
-    static constexpr int SLOT_LD = BQ + 4;                   // floats per receive-slot row (+4: spreads banks)
-    static constexpr int SLOT_BYTES = kBM * SLOT_LD * 4;     // split-K receive slots (all ranks' rows)
     static constexpr int ACC_COLS = BQ < 32 ? 32 : BQ;       // fp32 accumulator columns in TMEM
     static constexpr int SF_STRIDE = 32;                     // TMEM scale columns per stage: P 16, Q 16
     static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the 128-byte swizzle");
@@ -86,14 +83,15 @@ struct SkParams {
     int stages;            // ring depth, 1 .. kSkMaxStages
     int prefetch_w;        // the weights are constant: load them before waiting on the previous grid
     uint32_t tmem_cols;    // power of two >= 32
+    float4* ws;            // split-K partials: [tile][rank][BQ/4][128 rows] float4 (global workspace)
 };
 
-// Bytes of dynamic shared memory a launch needs: [ring][receive slots when
-// split][barriers][TMEM address, abort flag], 1024-byte aligned.
+// Bytes of dynamic shared memory a launch needs: [ring][barriers][TMEM
+// address, abort flag], 1024-byte aligned (the split-K partials meet in
+// global memory, so a split needs no more).
 template <int BQ>
-__host__ __device__ constexpr int sk_smem_bytes(int stages, bool split) {
-    return 1024 + stages * SkConfig<BQ>::STAGE_BYTES + (split ? SkConfig<BQ>::SLOT_BYTES : 0) +
-           8 * (4 * kSkMaxStages + 2) + 16;
+__host__ __device__ constexpr int sk_smem_bytes(int stages, [[maybe_unused]] bool split) {
+    return 1024 + stages * SkConfig<BQ>::STAGE_BYTES + 8 * (4 * kSkMaxStages + 2) + 16;
 }
 
 template <int BQ, bool SWAP>
@@ -106,9 +104,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = prm.stages;
     const int splits = gridDim.x;
-    // [ring][receive slots when split][barriers][tmem slot, abort flag]
+    // [ring][barriers][tmem slot, abort flag]
     const int ring_bytes = S * C::STAGE_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes + (splits > 1 ? C::SLOT_BYTES : 0));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * kSkMaxStages + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -125,7 +123,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     auto tfull_bar = [&](int s) { return bar_base + 8u * (kSkMaxStages + s); };
     auto empty_bar = [&](int s) { return bar_base + 8u * (2 * kSkMaxStages + s); };
     const uint32_t accum_bar = bar_base + 8u * (4 * kSkMaxStages);
-    const uint32_t red_bar = bar_base + 8u * (4 * kSkMaxStages + 1);
     auto stage_addr = [&](int s) { return smem_base + (uint32_t)(s * C::STAGE_BYTES); };
 
     if (threadIdx.x == 0) {
@@ -135,10 +132,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(accum_bar, 1);
-        mbar_init(red_bar, 1);
-        // Split: this CTA owns 128 / splits rows of the tile and receives them
-        // from every rank: 128 / splits * splits = 128 rows of BQ floats.
-        if (splits > 1) mbar_arrive_expect_tx(red_bar, (uint32_t)(kBM * BQ * 4));
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -156,7 +149,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (splits > 1) cluster_arrive_relaxed();   // "this CTA's barriers exist" (waited on before the first push)
     grid_launch_dependents();
 
     // Which operand holds the weights: P when swapped, Q otherwise.  Byte
@@ -300,8 +292,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     } else {
         const int quad = warp & 3;   // TMEM lane quadrant of this warp
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
-        grid_dependency_wait();   // before the D stores
-        if (splits > 1) cluster_wait();   // every peer's barriers exist (long done by now)
+        grid_dependency_wait();   // before the D stores and the split-K partials
         int acc_ok = 1;
         if (lane == 0) acc_ok = mbar_wait(accum_bar, 0, abort_flag) ? 1 : 0;
         acc_ok = __shfl_sync(0xffffffffu, acc_ok, 0);
@@ -359,113 +350,49 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     }
 
     if (splits > 1) {
-        // ---- split-K: partial rows to their owners, then the owners' sums
-        if (warp < 2) cluster_wait();   // pairs with the arrive at the start (epilogue warps waited above)
-        constexpr int LD = C::SLOT_LD;
-        const uint32_t slots = smem_base + (uint32_t)ring_bytes;
-        const int rows_per = kBM / splits;
-        if (warp >= 2) {
-            if (!*abort_flag) {
-                // Row `row` of this CTA's partial goes to rank row / rows_per,
-                // into slot `split` there: 16-byte asynchronous stores, each
-                // counted on the owner's red barrier.
-                const int quad = warp & 3;
-                const int row = quad * 32 + lane;
-                const uint32_t owner = (uint32_t)(row / rows_per);
-                const uint32_t local = slots + (uint32_t)((split * rows_per + row % rows_per) * LD) * 4u;
-                const uint32_t dst = cluster_rank_addr(local, owner);
-                const uint32_t dst_bar = cluster_rank_addr(red_bar, owner);
-                const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
-                // Up to 32 columns per TMEM load and one wait per 32: the
-                // loads' latency is paid once, not per 16 columns.
-                constexpr int CW = BQ < 32 ? BQ : 32;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BQ; c0 += CW) {
-                    uint32_t r[32];
-                    if (CW == 32) {
-                        tmem_load_32(t_quad + c0, r);
-                    } else {
-                        uint32_t h[16];
-                        tmem_load_16(t_quad + c0, h);
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) r[c] = h[c];
-                    }
-                    tmem_wait_load();
-#pragma unroll
-                    for (int c = 0; c < CW; c += 4)
-                        st_async_v4(dst + 4u * (c0 + c), r[c], r[c + 1], r[c + 2], r[c + 3], dst_bar);
-                }
-            }
-            // Wait for every rank's rows of this CTA (bounded: a rank that
-            // aborted sends nothing, and the wait then gives up).
-            int got = 1;
-            if (lane == 0) got = mbar_wait(red_bar, 0, abort_flag) ? 1 : 0;
-            got = __shfl_sync(0xffffffffu, got, 0);
-            if (!got) *abort_flag = 1;
-        }
-        __syncthreads();   // the owner's four warps have all seen the red barrier (or an abort)
+        // ---- split-K through L2: this CTA's fp32 partial tile -> the workspace
+        // (coalesced 16-byte stores), one cluster barrier (release/acquire at
+        // cluster scope orders them), then each rank sums its 128 / splits rows
+        // of every rank's partial in rank order -- the tiled kernel's exchange.
         if (warp >= 2 && !*abort_flag) {
-            // Owner `split` holds rows [split*rows_per, +rows_per) of the tile
-            // from every rank: slot z, row r at (z*rows_per + r)*LD floats.
+            const int quad = warp & 3;
+            const int row = quad * 32 + lane;
+            float4* dst = prm.ws + ((size_t)blockIdx.y * gridDim.x + split) * (size_t)(BQ / 4) * kBM;
+            const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+            constexpr int CW = BQ < 32 ? 16 : 32;   // columns per TMEM load (one wait each)
+#pragma unroll 1
+            for (int c0 = 0; c0 < BQ; c0 += CW) {
+                uint32_t r[32];
+                if (CW == 32) {
+                    tmem_load_32(t_quad + c0, r);
+                } else {
+                    uint32_t h[16];
+                    tmem_load_16(t_quad + c0, h);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) r[c] = h[c];
+                }
+                tmem_wait_load();
+#pragma unroll
+                for (int c = 0; c < CW / 4; ++c)
+                    dst[(c0 / 4 + c) * kBM + row] = make_float4(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1]),
+                                                                __uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3]));
+            }
+        }
+        cluster_sync();   // every rank's partial is in the workspace and visible to the cluster
+        if (warp >= 2 && !*abort_flag) {
+            GemmParams gp{};
+            gp.ws = prm.ws;
+            gp.D = prm.D;
+            gp.alpha = prm.alpha;
+            gp.rows_p = prm.rows_p;
+            gp.rows_q = prm.rows_q;
+            gp.ldd = prm.ldd;
             const int t = threadIdx.x - 64;
-            const int row0 = split * rows_per;
-            const uint32_t zstride = (uint32_t)(rows_per * LD) * 4u;
-            if (SWAP) {
-                // Thread -> (token column m, weight row r) of the owned
-                // rows, 8 consecutive r in 8 consecutive lanes; each sums its
-                // element over the ranks, then lane r % 8 == 0 gathers the 8
-                // sums of its group and writes D[m][n .. n+7] (16 bytes).
-                const int elems = BQ * rows_per;   // a multiple of 128 when rows_per >= 8 and BQ >= 16
-                for (int e = t; e < elems; e += 128) {
-                    const int r = e % rows_per, m_l = e / rows_per;
-                    float acc = 0.f;
-                    for (int z = 0; z < splits; ++z) {   // rank order
-                        float x;
-                        asm volatile("ld.shared.f32 %0, [%1];"
-                                     : "=f"(x)
-                                     : "r"(slots + z * zstride + (uint32_t)(r * LD + m_l) * 4u));
-                        acc += x;
-                    }
-                    const float o = acc * prm.alpha;
-                    float g[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) g[j] = __shfl_sync(0xffffffffu, o, (lane & ~7) | j);
-                    const int m = q_row0 + m_l, n = tp * kBM + row0 + r;
-                    if ((r & 7) == 0 && m < prm.rows_q && n < prm.rows_p) {
-                        uint4 w;
-                        w.x = pack_bf16x2(g[0], g[1]);
-                        w.y = pack_bf16x2(g[2], g[3]);
-                        w.z = pack_bf16x2(g[4], g[5]);
-                        w.w = pack_bf16x2(g[6], g[7]);
-                        *reinterpret_cast<uint4*>(prm.D + (size_t)m * prm.ldd + n) = w;
-                    }
-                }
-            } else {
-                // Item: one token row m and 8 consecutive weight columns n.
-                const int items = rows_per * (BQ / 8);
-                for (int it = t; it < items; it += 128) {
-                    const int r = it / (BQ / 8), c8 = it % (BQ / 8);
-                    float acc[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-                    for (int z = 0; z < splits; ++z) {   // rank order
-                        const uint32_t base = slots + z * zstride + (uint32_t)(r * LD + c8 * 8) * 4u;
-                        const uint4 a = ld_shared_v4(base), b = ld_shared_v4(base + 16);
-                        acc[0] += __uint_as_float(a.x), acc[1] += __uint_as_float(a.y);
-                        acc[2] += __uint_as_float(a.z), acc[3] += __uint_as_float(a.w);
-                        acc[4] += __uint_as_float(b.x), acc[5] += __uint_as_float(b.y);
-                        acc[6] += __uint_as_float(b.z), acc[7] += __uint_as_float(b.w);
-                    }
-                    const int m = tp * kBM + row0 + r, n = q_row0 + c8 * 8;
-                    if (m < prm.rows_p && n < prm.rows_q) {   // rows_q (= N) is a multiple of 8
-                        uint4 w;
-                        w.x = pack_bf16x2(acc[0] * prm.alpha, acc[1] * prm.alpha);
-                        w.y = pack_bf16x2(acc[2] * prm.alpha, acc[3] * prm.alpha);
-                        w.z = pack_bf16x2(acc[4] * prm.alpha, acc[5] * prm.alpha);
-                        w.w = pack_bf16x2(acc[6] * prm.alpha, acc[7] * prm.alpha);
-                        *reinterpret_cast<uint4*>(prm.D + (size_t)m * prm.ldd + n) = w;
-                    }
-                }
+            switch (splits) {
+                case 2: reduce_from_workspace<BQ, SWAP, 2>(gp, tp, q_row0, t); break;
+                case 4: reduce_from_workspace<BQ, SWAP, 4>(gp, tp, q_row0, t); break;
+                case 8: reduce_from_workspace<BQ, SWAP, 8>(gp, tp, q_row0, t); break;
+                default: reduce_from_workspace<BQ, SWAP, 16>(gp, tp, q_row0, t); break;
             }
         }
     }
