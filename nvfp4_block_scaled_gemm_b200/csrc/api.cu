@@ -620,10 +620,11 @@ nvfp4_status gemv_gemm(DeviceInfo* info, const void* A, const void* sA, const vo
     prm.prefetch_b = (flags & NVFP4_GEMM_B_CONSTANT) ? 1 : 0;
     int rw = M == 1 ? (N >= 2048 ? 4 : 1) : 2;
     if (use_gemv_areg(M, K)) {
-        // measured (us, 1 row): 2048 x 6144 rw2 2.53 / rw4 2.68; 8192 x 8192
-        // rw4 8.16 / rw2 8.27; 768 x 6144 rw1 1.94 / rw2 2.11.  Two rows:
-        // 256 x 6144 rw1 2.16 / rw2 2.39; 8192 x 8192 rw4 13.1 / rw2 14.6.
-        rw = N >= 4096 ? 4 : (M == 1 ? (N >= 2048 ? 2 : 1) : (N <= 256 ? 1 : 2));
+        // measured (us, 1 row): 2048 x 6144 rw4 2.55-2.68 / rw2 2.53-3.07
+        // (four runs); 8192 x 8192 rw4 7.73 / rw2 8.65; 768 x 6144 rw1 1.82 /
+        // rw2 1.99.  Two rows: 256 x 6144 rw1 2.16 / rw2 2.38; 2048 x 6144
+        // rw2 4.03 / rw4 4.90; 8192 x 8192 rw4 12.7 / rw2 12.4-14.6.
+        rw = M == 1 ? (N >= 2048 ? 4 : 1) : (N >= 4096 ? 4 : (N <= 256 ? 1 : 2));
     }
     if (const char* e = std::getenv("NVFP4_GEMM_GEMV_RW")) {
         const int v = std::atoi(e);

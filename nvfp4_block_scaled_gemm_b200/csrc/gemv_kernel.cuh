@@ -116,13 +116,23 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
     return (b & 0x80u) ? -v : v;
 }
 
+// The two halves of an f16x2 summed in fp32 (exact for these sums): the low
+// half converted, the high half added to it by a mixed f16 + f32 add.
+__device__ __forceinline__ float half2_sum_f32(__half2 s) {
+    const float lo = __low2float(s);
+    const unsigned short hi = __half_as_ushort(__high2half(s));
+    float r;
+    asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(r) : "h"(hi), "f"(lo));
+    return r;
+}
+
 // Exact sum of the 16 products of one block: 8 f16x2 of each operand.
 __device__ __forceinline__ float block_dot(const uint32_t* a, const uint32_t* b) {
     __half2 s = __hmul2(*reinterpret_cast<const __half2*>(&a[0]), *reinterpret_cast<const __half2*>(&b[0]));
 #pragma unroll
     for (int i = 1; i < 8; ++i)
         s = __hfma2(*reinterpret_cast<const __half2*>(&a[i]), *reinterpret_cast<const __half2*>(&b[i]), s);
-    return __low2float(s) + __high2float(s);
+    return half2_sum_f32(s);
 }
 
 // Sum NV per-thread values over the warp.  Each step halves the values a

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_sp24_kernel(const Gem
                                 for (int i = 1; i < 4; ++i)
                                     s2 = __hfma2(*reinterpret_cast<const __half2*>(&a[i]),
                                                  *reinterpret_cast<const __half2*>(&w[i]), s2);
-                                bsum[h] = __low2float(s2) + __high2float(s2);
+                                bsum[h] = half2_sum_f32(s2);
                             }
                             acc[r][m] = fmaf(bsum[0], sa0 * sb0[r], acc[r][m]);
                             acc[r][m] = fmaf(bsum[1], sa1 * sb1[r], acc[r][m]);
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kGemvThreads) nvfp4_gemv_sp24_areg_kernel(cons
                             for (int i = 1; i < 4; ++i)
                                 s2 = __hfma2(*reinterpret_cast<const __half2*>(&a[i]),
                                              *reinterpret_cast<const __half2*>(&w[i]), s2);
-                            bsum[h] = __low2float(s2) + __high2float(s2);
+                            bsum[h] = half2_sum_f32(s2);
                         }
                         acc[r][m] = fmaf(bsum[0], sa[m][j][0] * sb.x, acc[r][m]);
                         acc[r][m] = fmaf(bsum[1], sa[m][j][1] * sb.y, acc[r][m]);
