@@ -460,6 +460,23 @@ def source_hash() -> str:
     return h()
 
 
+def gpu_local_cpus(local_rank):
+    """The host CPUs NVML reports as closest to this GPU (its NUMA node), or
+    None.  Pinned host buffers allocated by a thread running there sit in that
+    node's memory, which is what the PCIe copies read."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(local_rank)
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, 16)   # 16 x 64-bit masks
+        cpus = {64 * i + b for i, w in enumerate(words) for b in range(64) if (w >> b) & 1}
+        pynvml.nvmlShutdown()
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
 def run_e2e(nv, torch, dev, base, steps, stream):
     """Same metric through nvfp4_gemm with pinned HOST buffers: every step copies
     all its inputs host->device (one pinned arena holding the six GEMMs' A, sA,
@@ -469,6 +486,18 @@ def run_e2e(nv, torch, dev, base, steps, stream):
     def pad(n):
         return (n + 255) // 256 * 256
 
+    # run (and allocate the pinned arenas) on the GPU's own NUMA node; restored below
+    saved_cpus = os.sched_getaffinity(0)
+    local = gpu_local_cpus(dev.index or 0)
+    if local:
+        os.sched_setaffinity(0, local)
+    try:
+        return _run_e2e(nv, torch, dev, base, steps, stream, pad, local)
+    finally:
+        os.sched_setaffinity(0, saved_cpus)
+
+
+def _run_e2e(nv, torch, dev, base, steps, stream, pad, local):
     # input arena: per GEMM A, sA, B, sB as bytes, each on a 256-byte boundary
     layout, off = [], 0
     for (m, ca, sa, cb, sb, al) in base:
@@ -519,7 +548,8 @@ def run_e2e(nv, torch, dev, base, steps, stream):
         assert torch.equal(h_out[oo:oo + m * N].view(m, N).view(torch.int16), dD.cpu().view(torch.int16))
     return {"value": round(step_bytes() * steps / (ms / 1e3) / 1e9, 3), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "copies_per_step": {"h2d": 1, "d2h": 1, "arena_bytes": int(off)}}
+            "copies_per_step": {"h2d": 1, "d2h": 1, "arena_bytes": int(off)},
+            "host_cpus": f"the GPU's NUMA-local CPUs ({len(local)})" if local else "all (NVML affinity unavailable)"}
 
 
 # ---------------------------------------------------------------- reference arm
