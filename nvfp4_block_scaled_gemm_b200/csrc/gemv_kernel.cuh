@@ -350,9 +350,11 @@ __device__ __forceinline__ float2 e4m3x2_values(uint32_t two) {
     return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// Resident CTAs per SM asked of the register allocator: two token rows
-// (64 registers of decoded chunks) four, or three with 4-row groups; one row
-// five, up to two chunks per thread.
+// Resident CTAs per SM asked of the register allocator (__launch_bounds__
+// minimum): two token rows (64 registers of decoded chunks) four, or three
+// with 4-row groups; one row with up to two chunks per thread four (the
+// 4-row form then takes 94 registers, so five fit; asking for five made it
+// spill).
 template <int MT, int RW, int CPT>
 constexpr int gemv_areg_min_ctas() {
     return MT == 2 ? (RW * CPT >= 8 ? 3 : 4) : (CPT <= 2 ? 4 : 1);
