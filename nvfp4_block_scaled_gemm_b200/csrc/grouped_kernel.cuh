@@ -20,9 +20,10 @@
 // unit descriptors in shared memory (job_full / job_empty barriers).
 //
 // Warp roles (320 threads): warp 0 TMA producer; warp 1 TMEM allocator and
-// MMA issuer; warps 2..5 epilogue (TMEM -> alpha[g] -> BF16 -> D); warps 6..9
-// scale writers (shared memory -> TMEM, one warp per lane quadrant, as in the
-// single GEMM kernel).  The fp32 accumulator is double-buffered in TMEM so the
+// MMA issuer; warps 2..5 epilogue (TMEM -> alpha[g] -> BF16, transposed
+// through shared memory into 16-byte stores to D); warps 6..9 scale writers
+// (shared memory -> TMEM, one warp per lane quadrant, as in the single GEMM
+// kernel).  The fp32 accumulator is double-buffered in TMEM so the
 // epilogue of one pass overlaps the main loop of the next.
 #pragma once
 
@@ -52,11 +53,12 @@ struct GroupedConfig {
     static constexpr int SFP_BYTES = 4 * kAtomBytes;
     static constexpr int SFQ_BYTES = 4 * kAtomBytes;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES + SFP_BYTES + SFQ_BYTES;
-    static constexpr int STAGES_FIT = (kSmemLimit - 2048) / STAGE_BYTES;
+    static constexpr int TAIL_BYTES = 1024 + 2 * kOrderMax;     // barriers, job ring, expert order
+    static constexpr int EPI_BYTES = 4 * 1024;                    // per epilogue warp: 16 token rows x 32 bf16
+    static constexpr int STAGES_FIT = (kSmemLimit - 1024 - TAIL_BYTES - EPI_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
     static_assert(STAGES >= kScaleBuffers, "scale buffers are released through the ring barriers");
-    static constexpr int TAIL_BYTES = 1024 + 2 * kOrderMax;     // barriers, job ring, expert order
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TAIL_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TAIL_BYTES + EPI_BYTES;
     // TMEM: two accumulators [0,BQ) and [BQ,2BQ), then 4 scale buffers of 32.
     static constexpr int ACC_COLS = BQ;
     static constexpr int SF_BASE = 2 * BQ;
@@ -306,12 +308,13 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         // ---- epilogue (warps 2..5, TMEM lane quadrant w % 4 = weight rows)
         const int quad = warp & 3;
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t epi = smem_addr(tail) + (uint32_t)(C::TAIL_BYTES + quad * 1024);
         int jc = 0;
         bool live = true;
         UnitJob jb;
         for (int j = 0; live && take_job(j, jb, true); ++j) {
             const float alpha = __ldg(prm.alpha + jb.g);
-            const int n = jb.nt * kBM + quad * 32 + lane;     // output column
+            const int n_warp = jb.nt * kBM + quad * 32;       // this warp's first output column
             for (int pass = 0; pass < jb.passes(); ++pass, ++jc) {
                 const int acc = jc & 1;
                 int ok = 1;
@@ -327,13 +330,26 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
                     uint32_t r[16];
                     tmem_load_16(t_quad + acc * C::ACC_COLS + c0, r);
                     tmem_wait_load();
-                    if (n < prm.N) {
+                    // Transpose through this warp's 1 KB of shared memory: row c
+                    // holds the 32 columns of token row q0 + c0 + c, which then
+                    // leave as 16-byte pieces of 8 consecutive columns.
 #pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            if (c0 + c < nq)
-                                prm.D[(size_t)(q0 + c0 + c) * prm.N + n] =
-                                    __float2bfloat16_rn(__uint_as_float(r[c]) * alpha);
+                    for (int c = 0; c < 16; ++c) {
+                        const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(r[c]) * alpha);
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(epi + (uint32_t)(c * 64 + lane * 2)),
+                                     "h"(*reinterpret_cast<const uint16_t*>(&h))
+                                     : "memory");
                     }
+                    __syncwarp();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int idx = lane + 32 * h, c = idx >> 2, part = idx & 3;
+                        const int n0 = n_warp + part * 8;   // N is a multiple of 8
+                        const uint4 val = ld_shared_v4(epi + (uint32_t)(c * 64 + part * 16));
+                        if (c0 + c < nq && n0 < prm.N)
+                            *reinterpret_cast<uint4*>(prm.D + (size_t)(q0 + c0 + c) * prm.N + n0) = val;
+                    }
+                    __syncwarp();
                 }
                 tc_fence_before();
                 __syncwarp();
