@@ -16,22 +16,25 @@
 // of A and runs MMAs with N = that many rows rounded up to 16 (the instruction
 // descriptor is built at run time).  Empty experts are never handed out.
 //
-// The producer passes each unit to the other roles through a small ring of
-// unit descriptors in shared memory (job_full / job_empty barriers).
+// The weight producer passes each unit to the other roles through a small ring
+// of unit descriptors in shared memory (job_full / job_empty barriers).
 //
-// Warp roles (320 threads): warp 0 TMA producer; warp 1 TMEM allocator and
-// MMA issuer; warps 2..5 epilogue (TMEM -> alpha[g] -> BF16, transposed
-// through shared memory into 16-byte stores to D); warps 6..9 scale writers
-// (shared memory -> TMEM, one warp per lane quadrant, as in the single GEMM
-// kernel).  The fp32 accumulator is double-buffered in TMEM so the
-// epilogue of one pass overlaps the main loop of the next.
+// Warp roles (352 threads): warp 0 weight producer (TMA of the weight tile and
+// its scales); warp 10 token producer (TMA of the unit's token rows and their
+// scales into the same ring stage: with every copy issued from one thread the
+// stream stalls on issue); warp 1 TMEM allocator and MMA issuer; warps 2..5
+// epilogue (TMEM -> alpha[g] -> BF16, transposed through shared memory into
+// 16-byte stores to D); warps 6..9 scale writers (shared memory -> TMEM, one
+// warp per lane quadrant, as in the single GEMM kernel).  The fp32
+// accumulator is double-buffered in TMEM so the epilogue of one pass overlaps
+// the main loop of the next.
 #pragma once
 
 #include "gemm_kernel.cuh"
 
 namespace nvfp4 {
 
-constexpr int kGroupedThreads = 320;
+constexpr int kGroupedThreads = 352;
 constexpr int kGroupedBQ = 128;   // max tokens per pass
 constexpr int kJobSlots = 4;      // unit descriptors in flight between the producer and the other roles
 constexpr int kOrderMax = 2048;   // experts ordered heavy-first in shared memory (natural order beyond)
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 1);
+            mbar_init(full_bar(s), 2);   // weight producer and token producer
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < NB; ++b) mbar_init(sf_ready_bar(b), 4);
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         }
         for (int j = 0; j < kJobSlots; ++j) {
             mbar_init(job_full_bar(j), 1);
-            mbar_init(job_empty_bar(j), 9);   // MMA issuer, 4 writer warps, 4 epilogue warps
+            mbar_init(job_empty_bar(j), 10);   // token producer, MMA issuer, 4 writer warps, 4 epilogue warps
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -182,7 +185,6 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
         __syncwarp();
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();   // each weight tile is read by one unit
-            const uint64_t pol_a = policy_evict_last();    // token rows are shared by all N tiles
             const unsigned total = (unsigned)listed * (unsigned)prm.tiles_n;
             auto describe = [&](unsigned u, UnitJob& jb) {
                 const int idx = (int)(u / (unsigned)prm.tiles_n);
@@ -219,9 +221,34 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
                         const int s = it % S;
                         if (!mbar_wait(empty_bar(s), ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag)) goto producer_done;
                         const uint32_t st = smem_base + s * C::STAGE_BYTES;
-                        mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + 16 * kBM + nbox * (16 * kStageKBytes + 16 * 16));
+                        mbar_arrive_expect_tx(full_bar(s), C::P_BYTES + 16 * kBM);
                         tma_load_2d(st, &tmB, full_bar(s), kt * kStageKBytes, brow, pol_w);
                         tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSB, full_bar(s), kt * 16, brow, pol_w);
+                    }
+                }
+            }
+        producer_done:;
+        }
+    } else if (warp == kGroupedThreads / 32 - 1) {
+        // ---- token producer: the unit's token rows and their scales, into
+        // the same ring stages (a second issuing thread: one thread issuing
+        // every copy of a stage limits the stream rate)
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_last();   // token rows are shared by all N tiles
+            int it = 0;
+            bool ok = true;
+            UnitJob jb;
+            for (int j = 0; ok && take_job(j, jb, false); ++j) {
+                for (int pass = 0; ok && pass < jb.passes(); ++pass) {
+                    const int nbox = (jb.q_rows(pass) + 15) / 16;
+                    for (int kt = 0; kt < prm.k_tiles; ++kt, ++it) {
+                        const int s = it % S;
+                        if (!mbar_wait(empty_bar(s), ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t st = smem_base + s * C::STAGE_BYTES;
+                        mbar_arrive_expect_tx(full_bar(s), nbox * (16 * kStageKBytes + 16 * 16));
                         for (int bx = 0; bx < nbox; ++bx) {
                             tma_load_2d(st + C::P_BYTES + bx * 16 * kStageKBytes, &tmA, full_bar(s), kt * kStageKBytes,
                                         jb.q_row0(pass) + 16 * bx, pol_a);
@@ -231,8 +258,8 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
                     }
                 }
             }
-        producer_done:;
         }
+        __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             int it = 0, jc = 0;
