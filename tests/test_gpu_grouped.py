@@ -48,6 +48,28 @@ def test_grouped_small_with_empty_and_large_groups(nv):
     assert not violations(got, ref, ad).any()
 
 
+@pytest.mark.parametrize("K", [1280, 2304])
+def test_grouped_every_box_count_and_partial_token_slots(nv, K):
+    # Passes of 1..8 sixteen-row boxes (MMA N = 16..128, row counts off a box
+    # edge too), two passes for one expert, K = 5 and 9 K tiles (not a
+    # multiple of the ring depth), and 384 weight rows: three units per
+    # expert, so the ring stages wrap around many times within one launch.
+    rng = np.random.default_rng(11)
+    N = 384
+    counts = [16 * b - (b % 3) for b in range(1, 9)] + [0, 200, 1, 33]
+    G = len(counts)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    Mt = int(off[-1])
+    A = synth.random_codes(Mt, K, 31)
+    sA = synth.random_scales(Mt, K, 32)
+    B = np.stack([synth.random_codes(N, K, 40 + g) for g in range(G)])
+    sB = np.stack([synth.random_scales(N, K, 60 + g) for g in range(G)])
+    alpha = rng.uniform(0.5, 2.0, G).astype(np.float32)
+    _, ref, ad = oracle.grouped_gemm(A, sA, B, sB, alpha, off, G, Mt, N, K)
+    got = run(nv, A, sA, B, sB, alpha, off)
+    assert not violations(got, ref, ad).any()
+
+
 def test_grouped_moe_recipe_reduced(nv):
     # The MoE recipe (Zipf routing, N(0,0.02) experts, N(0,1) tokens with 1%
     # x20 outliers, per-expert global scales) at N=256, K=1024, quantised by
