@@ -2,6 +2,7 @@
 
     python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes 512x768x6144 --iters 3
     python -m nvfp4_block_scaled_gemm_b200.profile_case --shapes attn --iters 2
+    python -m nvfp4_block_scaled_gemm_b200.profile_case --grouped 64 --iters 3
 
 `--traffic-csv FILE` (no GPU) instead turns the CSV log of an ncu run of
 `--shapes attn --iters 2` with the metrics gpu__time_duration.sum,
@@ -15,6 +16,12 @@ it was taken on.
 N=768, K=6144).  Inputs are seeded N(0,1) fp32 quantised on the GPU; every
 launch of a shape uses the same buffers (ncu flushes the caches between its
 replay passes, so DRAM counters still see the compulsory traffic).
+
+`--grouped E` runs the grouped MoE GEMM instead, on the MoE routing recipe
+(top-8, Zipf(1.1) popularity) with E experts of [2048 x 6144] and the tokens
+scaled with E (512 x E / 256), so experts keep about 16 rows each: E = 64
+keeps the device footprint near half a GB while the weights (0.4 GB) still
+exceed the L2, so a multi-pass ncu capture of the grouped kernel stays small.
 """
 from __future__ import annotations
 
@@ -90,6 +97,44 @@ def summarize_traffic(csv_path: str, out_path: str, iters: int = 2) -> dict:
     return out
 
 
+def run_grouped(experts: int, iters: int, seed: int):
+    import numpy as np
+
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    tokens = max(synth.MOE_TOPK, synth.MOE_TOKENS * experts // synth.MOE_EXPERTS)
+    r = synth.moe_routing(tokens=tokens, experts=experts)
+    Mt, N, K = int(r.row_offsets[-1]), synth.MOE_N, synth.HIDDEN_K
+    ct, st, ga = nv.quantize(torch.randn((tokens, K), generator=gen, device=dev))
+    tok = torch.from_numpy(r.token_of_row.astype(np.int64)).to(dev)
+    A, sA = ct[tok].contiguous(), st[tok].contiguous()
+    B = torch.empty((experts, N, K // 2), dtype=torch.uint8, device=dev)
+    sB = torch.empty((experts, N, K // 16), dtype=torch.uint8, device=dev)
+    alpha = torch.empty((experts,), dtype=torch.float32, device=dev)
+    for g in range(experts):
+        cb, sb, gb = nv.quantize(torch.randn((N, K), generator=gen, device=dev) * 0.02)
+        B[g].copy_(cb)
+        sB[g].copy_(sb)
+        alpha[g] = ga[0] * gb[0]
+    off = torch.from_numpy(r.row_offsets.astype(np.int32)).to(dev)
+    D = torch.empty((Mt, N), dtype=torch.bfloat16, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        nv.grouped_gemm(A, sA, B, sB, alpha, off, out=D)
+    e1.record()
+    torch.cuda.synchronize()
+    status = nv.get_device_error()
+    if status != 0:
+        raise SystemExit(f"device error status {status}")
+    counts = [int(c) for c in np.diff(r.row_offsets)]
+    us = e0.elapsed_time(e1) * 1e3 / iters
+    print(f"grouped {experts} experts x [{N} x {K}], {tokens} tokens top-{synth.MOE_TOPK} -> {Mt} rows "
+          f"({sum(c > 0 for c in counts)} active, at most {max(counts)} per expert): "
+          f"{us:.2f} us/launch (eager), {accounting.grouped_bytes(counts, N, K) / us / 1e3:.0f} GB/s algorithmic")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--shapes", default="512x768x6144")
@@ -97,9 +142,13 @@ def main():
     ap.add_argument("--seed", type=int, default=1)
     ap.add_argument("--traffic-csv", default=None, help="ncu CSV of `--shapes attn --iters 2` (pass --iters 2)")
     ap.add_argument("--traffic-out", default="profiles/traffic_attn_sweep.json")
+    ap.add_argument("--grouped", type=int, default=0, help="run the grouped MoE GEMM with this many experts")
     args = ap.parse_args()
     if args.traffic_csv:
         print(summarize_traffic(args.traffic_csv, args.traffic_out, args.iters))
+        return
+    if args.grouped:
+        run_grouped(args.grouped, args.iters, args.seed)
         return
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev)
