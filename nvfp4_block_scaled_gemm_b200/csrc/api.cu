@@ -259,7 +259,7 @@ int split_cluster_capacity(DeviceInfo* info, int splits) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3((unsigned)splits, 1, 1);
-        q.blockDim = dim3(nvfp4::kThreads, 1, 1);
+        q.blockDim = dim3(nvfp4::gemm_threads<BQ, SWAP, SFR, false>(), 1, 1);
         q.dynamicSmemBytes = C::SMEM_BYTES;
         cudaLaunchAttribute ca[1];
         ca[0].id = cudaLaunchAttributeClusterDimension;
@@ -388,7 +388,7 @@ nvfp4_status launch_gemm_kernel(DeviceInfo* info, uint64_t bit, const Maps& m, c
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(nvfp4::kThreads, 1, 1);
+    cfg.blockDim = dim3(nvfp4::gemm_threads<BQ, SWAP, SFR, QBF16>(), 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];

@@ -11,12 +11,14 @@
 // weights, Q = A, the few activation rows) so that the weight matrix streams
 // through the 128-row MMA side, and the epilogue writes the transpose.
 //
-// Warp roles (192 threads):
+// Warp roles (192 threads, 224 where gemm_two_producers holds):
 //   warp 0      TMA producer: per 256-element K tile, the P and Q operand
 //               tiles (2-D TMA, 128-byte swizzle) and their scales into a
 //               STAGES-deep shared-memory ring.  Scales arrive either as
 //               row-major [rows][16 B] tiles (SFR: one 2-D TMA box per
 //               operand) or already in 512-byte atoms (bulk copies).
+//   warp 6      (gemm_two_producers only) the Q tile and its scales, so
+//               that warp 0 issues only the P side.
 //   warp 1      TMEM allocator and MMA issuer: four
 //               tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 each) per K tile.
 //   warps 2..5  scale writers during the main loop, epilogue afterwards.  Warp
@@ -71,6 +73,23 @@ constexpr int kStageKBytes = 128; // = one 128-byte swizzle row of packed E2M1
 constexpr int kStepK = 64;        // K of one tcgen05.mma (mxf4nvf4, dense)
 constexpr int kAtomBytes = 512;   // scale atom: 128 rows x 4 blocks of 16
 constexpr int kThreads = 192;
+
+// Instantiations whose Q-side copies (tile and scales) come from a second
+// producer warp, warp 6: one thread issuing every copy of a stage delays the
+// stream when a stage's boxes are many or large.  Measured on graph-replayed
+// calls with constant weights (us, one producer -> two): 512 x 768 x 6144
+// (128-wide tiles) 9.63 -> 9.22, 512 x 2048 x 6144 12.79 -> 12.43, 4 and
+// 8 x 8192 x 8192 (16-row swapped tiles) 14.3 -> 13.4; the 64-wide tiles lost
+// about 1% (128 x 768, 256 x 2048) and the 32-row swapped tiles 0.05 us.
+template <int BQ, bool SWAP, bool SFR, bool QBF16>
+__host__ __device__ constexpr bool gemm_two_producers() {
+    return SFR && !QBF16 && ((!SWAP && BQ >= 128) || (SWAP && BQ == 16));
+}
+
+template <int BQ, bool SWAP, bool SFR, bool QBF16>
+__host__ __device__ constexpr int gemm_threads() {
+    return gemm_two_producers<BQ, SWAP, SFR, QBF16>() ? kThreads + 32 : kThreads;
+}
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 constexpr int kScaleBuffers = 4;    // rotating TMEM scale buffers
 
@@ -303,7 +322,7 @@ __device__ __forceinline__ void reduce_from_workspace(const GemmParams& prm, int
 // TMA box starts on a 16-byte boundary, so K tile kt loads the 16-byte box of
 // K tiles kt & ~1 and kt | 1, and the writers take its half kt % 2.
 template <int BQ, bool SWAP, bool SPLITK, bool SFR, bool QBF16 = false, bool MX = false>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<BQ, SWAP, SFR, QBF16>(), 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                       const GemmParams prm) {
@@ -312,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using C = TileConfig<BQ, SPLITK, QBF16>;
     constexpr int S = C::STAGES;
     constexpr int NB = kScaleBuffers;
+    constexpr bool TWO = gemm_two_producers<BQ, SWAP, SFR, QBF16>();   // warp 6 loads the Q side
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // [ring: S stages][split-K receive slots][barriers]
@@ -345,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 1);
+            mbar_init(full_bar(s), TWO ? 2 : 1);   // the producer warp(s)
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < NB; ++b) mbar_init(sf_ready_bar(b), 4);
@@ -373,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Everything above overlaps the previous kernel's tail when launched with
     // programmatic stream serialisation; global memory is touched only below.
     grid_launch_dependents();
-    const bool producer = (warp == 0 && lane == 0);
+    const bool producer = ((warp == 0 || (TWO && warp == 6)) && lane == 0);
     if (!producer) grid_dependency_wait();
 
     if (warp == 0) {
@@ -391,10 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto sf_x = [](int kt) { return MX ? 16 * (kt >> 1) : 16 * kt; };
             // With a constant B, its first ring's worth of tiles is requested
             // before waiting for the previous grid (only B is touched then).
-            // bytes of one stage: P tile + P scales + the Q side (FP4 tile and
-            // scales, or the raw BF16 tile that the writers quantize)
+            // bytes of one stage from this warp: P tile + P scales, and (one
+            // producer) the Q side: FP4 tile and scales, or the raw BF16 tile
+            // that the writers quantize
             constexpr uint32_t kStageTx =
-                C::P_BYTES + 16 * kBM + (QBF16 ? (uint32_t)C::QRAW_BYTES : (uint32_t)(C::Q_BYTES + 16 * BQ));
+                C::P_BYTES + 16 * kBM +
+                (TWO ? 0u : QBF16 ? (uint32_t)C::QRAW_BYTES : (uint32_t)(C::Q_BYTES + 16 * BQ));
             auto load_q = [&](uint32_t st, uint32_t bar, int kt) {
                 if (QBF16) {
                     tma_load_2d(st + C::QRAW_OFF, &tmQ, bar, kt * 256, q_row0, pol_q);
@@ -404,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             };
             int pre = 0;
-            if (SFR && prm.prefetch_b) {
+            if (SFR && prm.prefetch_b && (SWAP || !TWO)) {   // B is P, or this warp also loads Q = B
                 pre = min(S, kt_end - kt_begin);
                 for (int i = 0; i < pre; ++i) {
                     const int kt = kt_begin + i;
@@ -428,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t st = smem_base + s * C::STAGE_BYTES;
                 if (it < pre) {   // the other operand of a prefetched stage
                     if (SWAP) {
-                        load_q(st, full_bar(s), kt);
+                        if (!TWO) load_q(st, full_bar(s), kt);
                     } else {
                         tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
                         tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), sf_x(kt), tp * kBM, pol_p);
@@ -441,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(full_bar(s), kStageTx);
                     tma_load_2d(st, &tmP, full_bar(s), kt * kStageKBytes, tp * kBM, pol_p);
                     tma_load_2d(st + C::P_BYTES + C::Q_BYTES, &tmSP, full_bar(s), sf_x(kt), tp * kBM, pol_p);
-                    load_q(st, full_bar(s), kt);
+                    if (!TWO) load_q(st, full_bar(s), kt);
                 } else {
                     // atoms per 128-row block: one per K step (NVFP4) or per
                     // pair of K steps (MXFP4)
@@ -462,6 +484,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+    } else if (TWO && warp == 6) {
+        // ---- Q-side producer: the Q tile and its row-major scale box per K
+        // tile, on the same stage barriers (each stage expects both warps)
+        if (lane == 0) {
+            const uint64_t pol_q = policy_evict_last();
+            auto sf_x = [](int kt) { return MX ? 16 * (kt >> 1) : 16 * kt; };
+            constexpr uint32_t kQTx = C::Q_BYTES + 16 * BQ;
+            auto load_q = [&](int i, int kt) {
+                const uint32_t st = smem_base + (i % S) * C::STAGE_BYTES;
+                mbar_arrive_expect_tx(full_bar(i % S), kQTx);
+                tma_load_2d(st + C::P_BYTES, &tmQ, full_bar(i % S), kt * kStageKBytes, q_row0, pol_q);
+                tma_load_2d(st + C::P_BYTES + C::Q_BYTES + C::SFP_BYTES, &tmSQ, full_bar(i % S), sf_x(kt), q_row0,
+                            pol_q);
+            };
+            // a constant B on the Q side (not swapped): its first ring's worth
+            // of tiles before the wait for the previous grid
+            int pre = 0;
+            if (!SWAP && prm.prefetch_b) {
+                pre = min(S, kt_end - kt_begin);
+                for (int i = 0; i < pre; ++i) load_q(i, kt_begin + i);
+            }
+            grid_dependency_wait();
+            int it = pre;
+            for (int kt = kt_begin + pre; kt < kt_end; ++kt, ++it) {
+                if (!mbar_wait(empty_bar(it % S), ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag)) break;
+                load_q(it, kt);
+            }
+        }
+        __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_nvf4(kBM, BQ);
@@ -522,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(accum_bar);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 6) {
         const int quad = warp & 3;               // TMEM lane quadrant of this warp
         const uint32_t t_quad = tmem + ((uint32_t)(quad * 32) << 16);
         // ---- scale writers: shared memory -> TMEM scale buffer, per K tile.
@@ -683,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Partial tile -> workspace (after the grid dependency wait, which
         // every epilogue thread passed at the start), one cluster barrier,
         // then each owner's sum.
-        if (warp >= 2 && !*abort_flag) {
+        if (warp >= 2 && warp < 6 && !*abort_flag) {
             const int quad = warp & 3;
             const int row = quad * 32 + lane;
             float4* dst = partial_block<BQ>(prm, split);
@@ -708,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         cluster_sync();   // every rank's partial is in the workspace and visible to the cluster
-        if (warp >= 2 && !*abort_flag) {
+        if (warp >= 2 && warp < 6 && !*abort_flag) {
             const int t = threadIdx.x - 64;
             switch (splits) {
                 case 2: reduce_from_workspace<BQ, SWAP, 2>(prm, tp, q_row0, t); break;
