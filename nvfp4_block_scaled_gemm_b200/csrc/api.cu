@@ -310,7 +310,12 @@ Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr, int max_splits =
     }
     // Tile shape (measured on the attention and MoE decode shapes): weight
     // rows on the 128-row MMA side with narrow token tiles for small M, then
-    // 64- and 128-wide N tiles; 256-wide tiles once the grid is large.
+    // 64- and 128-wide N tiles; 256-wide tiles once the grid is large.  For
+    // 128 < M <= 256 the 128-wide tiles (which have the second producer warp)
+    // win once N >= 2048 (graph-replayed, constant weights, us: 256 x 2048 x
+    // 6144 11.0 -> 10.2, 256 x 4096 x 6144 16.2 -> 13.3, 256 x 6144 x 768
+    // 11.8 -> 7.5, 256 x 8192 x 8192 38.1 -> 23.8) and lose at N = 1024
+    // (8.25 -> 8.96); at N <= 768 the two are even.
     if (M <= 64) {
         p.swap = true;
         p.bq = M <= 16 ? 16 : 32;
@@ -320,7 +325,7 @@ Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr, int max_splits =
         if (N <= 256 && M > 256)
             p.bq = M <= 512 ? 32 : 64;   // few weight columns: more, narrower tiles
         else
-            p.bq = M <= 256 ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
+            p.bq = (M <= 128 || (M <= 256 && N < 2048)) ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
         // Without row-major scale tiles the scales of a Q tile come as whole
         // 128-row atoms, so a narrower Q tile is only possible alone.
         if (!sfr && p.bq < 128 && N > p.bq) p.bq = 128;

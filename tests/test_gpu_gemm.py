@@ -320,6 +320,17 @@ def test_config_shape_sampled(nv, monkeypatch, name, M, N, K, kind, seed, kernel
     assert not violations(got, ref, ad).any()
 
 
+# 128 < M <= 256 with N >= 2048 takes 128-wide tiles, which have the second
+# producer warp: full, ragged and short-K shapes on the default plan, sampled.
+@pytest.mark.parametrize("M,N,K", [(256, 8192, 8192), (256, 6144, 768), (200, 2048, 2048), (129, 4096, 1024)])
+def test_mid_m_wide_n_sampled(nv, M, N, K):
+    ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "normal", 71)
+    rows, cols = boundary_samples(M, N, 71, n_random=2000)
+    got = run_gemm_sampled(nv, ca, sa, cb, sb, alpha, rows, cols)
+    _, ref, ad = oracle.gemm_sampled(ca, sa, cb, sb, alpha, M, N, K, rows, cols)
+    assert not violations(got, ref, ad).any()
+
+
 # ------------------------------------------------------------------ bounded waits
 def test_wait_timeout_reports_and_context_survives(nv):
     assert nv.get_device_error() == 0
