@@ -308,14 +308,22 @@ Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr, int max_splits =
         // without row-major scale tiles, a narrow Q tile must start on a 128-row block
         if (sfr || p.bq >= 128 || p.tiles_q == 1) return p;
     }
+    // Split K over a cluster of up to 8 CTAs (a power of two, so that the 128
+    // tile rows divide evenly in the reduction) while the grid stays at or
+    // below ~128 CTAs, which leaves room for the next kernel's CTAs to start
+    // (programmatic dependent launch), and all of its clusters fit on the GPU
+    // at once.  (Clusters of 16 win for one shape timed alone but lose in a
+    // sequence of different shapes: they wait for whole free GPCs.)
+    const int cap = std::min(num_sms, 128);
+    auto splits_for = [&](int bq, int tiles) {
+        int splits = 1;
+        for (int s = 2; s <= max_splits && s <= p.k_tiles && tiles * s <= cap; s *= 2)
+            if (split_cluster_capacity_of(info, p.swap, bq, sfr, s) >= tiles) splits = s;
+        return splits;
+    };
     // Tile shape (measured on the attention and MoE decode shapes): weight
     // rows on the 128-row MMA side with narrow token tiles for small M, then
-    // 64- and 128-wide N tiles; 256-wide tiles once the grid is large.  For
-    // 128 < M <= 256 the 128-wide tiles (which have the second producer warp)
-    // win once N >= 2048 (graph-replayed, constant weights, us: 256 x 2048 x
-    // 6144 11.0 -> 10.2, 256 x 4096 x 6144 16.2 -> 13.3, 256 x 6144 x 768
-    // 11.8 -> 7.5, 256 x 8192 x 8192 38.1 -> 23.8) and lose at N = 1024
-    // (8.25 -> 8.96); at N <= 768 the two are even.
+    // 64- and 128-wide N tiles; 256-wide tiles once the grid is large.
     if (M <= 64) {
         p.swap = true;
         p.bq = M <= 16 ? 16 : 32;
@@ -325,25 +333,27 @@ Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr, int max_splits =
         if (N <= 256 && M > 256)
             p.bq = M <= 512 ? 32 : 64;   // few weight columns: more, narrower tiles
         else
-            p.bq = (M <= 128 || (M <= 256 && N < 2048)) ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
+            p.bq = M <= 256 ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
+        // 64-wide tiles for 64 < M <= 256, unless they would need more tiles
+        // than SMs or leave each CTA a stream of 12 or more K tiles: there the
+        // 128-wide tiles (which have the second producer warp) win.  Graph-
+        // replayed, constant weights, us (64-wide -> 128-wide): 96 x 8192 x
+        // 8192 33.6 -> 23.2, 128 x 8192 x 8192 21.7 -> 16.3, 128 x 4096 x 6144
+        // 11.9 -> 10.7, 256 x 2048 x 6144 11.0 -> 10.2, 256 x 6144 x 768
+        // 11.8 -> 7.5, 256 x 8192 x 8192 38.1 -> 23.8; with shorter streams
+        // the 64-wide tiles win or tie (128 x 2048 x 6144 8.5 against 9.2,
+        // 256 x 1024 x 6144 8.25 against 8.96, 256 x 768 x 6144 even).
+        if (sfr && p.bq == 64 && M <= 256) {
+            const int tiles64 = ((M + 127) / 128) * ((N + 63) / 64);
+            if (tiles64 > num_sms || p.k_tiles / splits_for(64, tiles64) >= 12) p.bq = 128;
+        }
         // Without row-major scale tiles the scales of a Q tile come as whole
         // 128-row atoms, so a narrower Q tile is only possible alone.
         if (!sfr && p.bq < 128 && N > p.bq) p.bq = 128;
     }
     p.tiles_p = p.swap ? (N + 127) / 128 : (M + 127) / 128;
     p.tiles_q = p.swap ? (M + p.bq - 1) / p.bq : (N + p.bq - 1) / p.bq;
-    // Split K over a cluster of up to 8 CTAs (a power of two, so that the 128
-    // tile rows divide evenly in the reduction) while the grid stays at or
-    // below ~128 CTAs, which leaves room for the next kernel's CTAs to start
-    // (programmatic dependent launch), and all of its clusters fit on the GPU
-    // at once.  (Clusters of 16 win for one shape timed alone but lose in a
-    // sequence of different shapes: they wait for whole free GPCs.)
-    const int tiles = p.tiles_p * p.tiles_q;
-    const int cap = std::min(num_sms, 128);
-    int splits = 1;
-    for (int s = 2; s <= max_splits && s <= p.k_tiles && tiles * s <= cap; s *= 2)
-        if (split_cluster_capacity_of(info, p.swap, p.bq, sfr, s) >= tiles) splits = s;
-    p.splits = splits;
+    p.splits = splits_for(p.bq, p.tiles_p * p.tiles_q);
     return p;
 }
 
