@@ -392,10 +392,12 @@ def test_gemm_b_constant_prefetch_matches_oracle(nv, M, N, K):
         assert not violations(D.float().cpu().numpy(), ref, ad).any()
 
 
-def test_gemm_b_constant_after_producer_of_A(nv):
+@pytest.mark.parametrize("M,N,K", [(8, 768, 2048), (16, 256, 1024), (512, 768, 2048)])
+def test_gemm_b_constant_after_producer_of_A(nv, M, N, K):
     # A is written by the kernel right before the GEMM; with the flag only B
-    # may be read early, so D must reflect the new A.
-    M, N, K = 8, 768, 2048
+    # may be read early, so D must reflect the new A.  The shapes take the
+    # split-K kernel, the swapped 16-row tiles and the 128-wide unswapped
+    # tiles (the last two with A and B on separate producer warps).
     ca, sa, cb, sb, alpha = quantized_problem(M, N, K, "normal", 91)
     ca2, sa2, _, _, _ = quantized_problem(M, N, K, "normal", 92)
     _, ref2, ad2 = oracle.gemm(ca2, sa2, cb, sb, alpha, M, N, K)
