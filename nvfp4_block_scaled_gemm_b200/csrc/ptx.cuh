@@ -138,17 +138,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank) 
         : "memory");
 }
 
-// 16-byte asynchronous store into the shared memory of another CTA of this
-// cluster (`addr` and `bar` are shared::cluster addresses, from mapa), whose
-// completion is counted in bytes on the mbarrier at `bar`.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     addr),
-                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
-                 : "memory");
-}
-
 // ------------------------------------------------------------ TMA and bulk
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
