@@ -334,18 +334,20 @@ Plan make_plan(int M, int N, int K, DeviceInfo* info, bool sfr, int max_splits =
             p.bq = M <= 512 ? 32 : 64;   // few weight columns: more, narrower tiles
         else
             p.bq = M <= 256 ? 64 : M <= 1024 ? 128 : (N >= 256 ? 256 : 128);
-        // 64-wide tiles for 64 < M <= 256, unless they would need more tiles
-        // than SMs or leave each CTA a stream of 12 or more K tiles: there the
-        // 128-wide tiles (which have the second producer warp) win.  Graph-
-        // replayed, constant weights, us (64-wide -> 128-wide): 96 x 8192 x
-        // 8192 33.6 -> 23.2, 128 x 8192 x 8192 21.7 -> 16.3, 128 x 4096 x 6144
-        // 11.9 -> 10.7, 256 x 2048 x 6144 11.0 -> 10.2, 256 x 6144 x 768
-        // 11.8 -> 7.5, 256 x 8192 x 8192 38.1 -> 23.8; with shorter streams
-        // the 64-wide tiles win or tie (128 x 2048 x 6144 8.5 against 9.2,
-        // 256 x 1024 x 6144 8.25 against 8.96, 256 x 768 x 6144 even).
-        if (sfr && p.bq == 64 && M <= 256) {
-            const int tiles64 = ((M + 127) / 128) * ((N + 63) / 64);
-            if (tiles64 > num_sms || p.k_tiles / splits_for(64, tiles64) >= 12) p.bq = 128;
+        // Tiles narrower than 128 (64 < M <= 256, or few weight columns),
+        // unless they would need more tiles than SMs or leave each CTA a
+        // stream of 12 or more K tiles: there the 128-wide tiles (which have
+        // the second producer warp) win.  Graph-replayed, constant weights,
+        // us (narrow -> 128-wide): 96 x 8192 x 8192 33.6 -> 23.2, 128 x 8192 x
+        // 8192 21.7 -> 16.3, 128 x 4096 x 6144 11.9 -> 10.7, 256 x 2048 x 6144
+        // 11.0 -> 10.2, 256 x 6144 x 768 11.8 -> 7.5, 256 x 8192 x 8192 38.1
+        // -> 23.8, 2048 x 256 x 6144 10.8 -> 9.9; with shorter streams the
+        // narrow tiles win or tie (128 x 2048 x 6144 8.5 against 9.2, 256 x
+        // 1024 x 6144 8.25 against 8.96, 256 x 768 x 6144 and 512 x 256 x 6144
+        // even).
+        if (sfr && p.bq < 128) {
+            const int tiles_n = ((M + 127) / 128) * ((N + p.bq - 1) / p.bq);
+            if (tiles_n > num_sms || p.k_tiles / splits_for(p.bq, tiles_n) >= 12) p.bq = 128;
         }
         // Without row-major scale tiles the scales of a Q tile come as whole
         // 128-row atoms, so a narrower Q tile is only possible alone.
