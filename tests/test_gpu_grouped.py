@@ -48,14 +48,15 @@ def test_grouped_small_with_empty_and_large_groups(nv):
     assert not violations(got, ref, ad).any()
 
 
-@pytest.mark.parametrize("K", [1280, 2304])
-def test_grouped_every_box_count_and_partial_token_slots(nv, K):
+@pytest.mark.parametrize("K,N", [(1280, 384), (2304, 200)])
+def test_grouped_every_box_count_and_ragged_k_tiles(nv, K, N):
     # Passes of 1..8 sixteen-row boxes (MMA N = 16..128, row counts off a box
     # edge too), two passes for one expert, K = 5 and 9 K tiles (not a
-    # multiple of the ring depth), and 384 weight rows: three units per
-    # expert, so the ring stages wrap around many times within one launch.
+    # multiple of the ring depth), and N = 384 weight rows (three units per
+    # expert), so the ring stages wrap around many times within one launch.
+    # N = 200 ends in a 72-column weight tile: the epilogue's 16-byte pieces
+    # stop inside the third lane quadrant.
     rng = np.random.default_rng(11)
-    N = 384
     counts = [16 * b - (b % 3) for b in range(1, 9)] + [0, 200, 1, 33]
     G = len(counts)
     off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
