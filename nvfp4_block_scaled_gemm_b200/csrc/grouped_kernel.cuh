@@ -314,10 +314,12 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
                 const int s = it % S, b = it % NB, jj = it - NB;
                 int got = 1;
                 // scale buffer b was last used by K tile it - NB, released by
-                // the MMA commit on that tile's ring stage
+                // the MMA commit on that tile's ring stage; with one buffer per
+                // stage that is stage s's previous phase, which the producer
+                // waited for before the loads that full(s) reports
                 if (lane == 0)
                     got = mbar_wait(full_bar(s), (uint32_t)(it / S) & 1u, abort_flag) &&
-                          (jj < 0 || mbar_wait(empty_bar(jj % S), (uint32_t)(jj / S) & 1u, abort_flag));
+                          (NB == S || jj < 0 || mbar_wait(empty_bar(jj % S), (uint32_t)(jj / S) & 1u, abort_flag));
                 if (!__shfl_sync(0xffffffffu, got, 0)) {
                     ok = false;
                     break;
